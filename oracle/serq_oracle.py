@@ -1,0 +1,419 @@
+"""SERQ CPU oracle — TEST INFRASTRUCTURE ONLY.
+
+A plain, slow, step-by-step CPU restatement of what the SERQ W4A4 linear
+computes.  Only the tests, the package's ``smoke()`` self-check and the
+benchmark's CPU-baseline leg may import it; the library path never does.
+It shares no code with the CUDA path.
+
+Sources (cited by page title and section):
+  [notes]   "SERQ: Saliency-Aware Low-Rank Error Reconstruction for LLM
+            Quantization" reading notes (dihengye.cn): 关键公式/基础量化,
+            Stage 1 (SAF), Stage 2 (saliency-aware error reconstruction),
+            量化推理 (quantized inference), Stage 3 (offline permutation).
+  [gist-zh] technical summary (gist.science/zh): 2.1 静态激活展平,
+            2.2 显著性感知误差重建, 2.3 离线权重置换, 3 主要贡献.
+  [gist-pt] resumo técnico (gist.science/pt): 2. Metodologia items 1-3.
+  [MX]      OCP Microscaling Formats (MX) Specification v1.0 — the pages only
+            name MXFP4; its element (E2M1) and shared-scale (E8M0) rules come
+            from this public specification.
+
+Arithmetic conventions (the pages fix none of them; these are the readings
+used everywhere in this repository):
+  * every quantization decision is taken in IEEE float32 with one rounding
+    per operation and no fused multiply-add: s = fp32(amax / 7),
+    q = rne(fp32(x / s)) -- numpy float32 ops round exactly this way;
+  * round-half-to-even for the INT4 grid and for E2M1 (ties go to the even
+    code);
+  * products are exact (small integers, or E2M1 values times powers of two),
+    accumulated in int64-exact float64 (INT4) or float64 (MXFP4).
+
+Parity pins: every function here is pinned by tests under tests/ against
+closed forms, hand cases, invariants (r=0 is plain W4A4, R=0 when the salient
+rows are on the grid, SAF/permutation identity, permutation invariance) and a
+brute-force dequantize-then-loop matmul on tiny shapes.  The choice among the
+readings of which Q(W_s) the residual subtracts, how the salient activation
+slice is scaled, and how the SAF calibration set is drawn cannot be pinned by
+any value the pages print (parity unpinned for those readings; the
+computation under each reading is pinned).
+"""
+
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+F32 = np.float32
+INT4_QMAX = 7                       # 2^(n-1) - 1 with n = 4  [notes, 基础量化]
+MX_BLOCK = 32                       # elements sharing one E8M0 scale  [MX]
+E2M1_EMAX = 2                       # exponent of the largest E2M1 normal (6 = 1.5 * 2^2)  [MX]
+E8M0_BIAS = 127                     # [MX]
+E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])  # magnitudes of codes 0..7  [MX]
+
+
+# ---------------------------------------------------------------------------
+# rounding helpers
+# ---------------------------------------------------------------------------
+
+def bf16_rne(x: np.ndarray) -> np.ndarray:
+    """float32 -> nearest bfloat16 (ties to even), returned as float32."""
+    x = np.ascontiguousarray(x, dtype=F32)
+    assert np.all(np.isfinite(x)), "non-finite input"
+    u = x.view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
+    return (u.astype(np.uint32) << 16).view(F32)
+
+
+# ---------------------------------------------------------------------------
+# A1: symmetric absmax INT4 quantizer  [notes, 基础量化]
+#     X_q = clip(round(X / s)),  s = max|X| / (2^(n-1) - 1)
+# ---------------------------------------------------------------------------
+
+def int4_scale(absmax: np.ndarray) -> np.ndarray:
+    """s = fp32(max|X| / 7)."""
+    return (np.asarray(absmax, dtype=F32) / F32(INT4_QMAX)).astype(F32)
+
+
+def int4_codes(x: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """q = clip(rne(fp32(x / s)), -7, 7); all-zero codes where s == 0."""
+    x = np.asarray(x, dtype=F32)
+    s = np.asarray(s, dtype=F32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        v = (x / s).astype(F32)
+    q = np.rint(v)
+    q = np.where(s > 0, q, 0.0)
+    return np.clip(q, -INT4_QMAX, INT4_QMAX).astype(np.int8)
+
+
+def quantize_int4(x: np.ndarray, axis: int):
+    """Per-slice symmetric INT4 along ``axis``: returns (codes int8, scale fp32)."""
+    x = np.asarray(x, dtype=F32)
+    s = int4_scale(np.max(np.abs(x), axis=axis, keepdims=True))
+    return int4_codes(x, s), np.squeeze(s, axis=axis)
+
+
+# ---------------------------------------------------------------------------
+# A12: MXFP4 = E2M1 elements + one E8M0 scale per 32 elements  [MX]
+# ---------------------------------------------------------------------------
+
+def mx_scale_exponent(absmax: np.ndarray) -> np.ndarray:
+    """Shared exponent E = floor(log2(absmax)) - emax(E2M1), clamped to [-127, 127].
+
+    absmax == 0 gives E = -127 (the smallest scale; all codes are then 0).
+    """
+    a = np.asarray(absmax, dtype=np.float64)
+    _, ex = np.frexp(a)                       # a = m * 2^ex, m in [0.5, 1)
+    e = ex.astype(np.int64) - 1 - E2M1_EMAX   # floor(log2 a) = ex - 1
+    e = np.where(a > 0, e, -E8M0_BIAS)
+    return np.clip(e, -E8M0_BIAS, E8M0_BIAS).astype(np.int32)
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 code for already-scaled values (ties to the even code).
+
+    The magnitude is the grid point closest to |v| (values past 6 take 6, the
+    largest finite E2M1 value); when |v| sits exactly half-way between two grid
+    points the even code wins.  The sign bit is the IEEE sign bit of v.
+    """
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    flat = a.reshape(-1)
+    mag = np.empty(flat.shape, dtype=np.uint8)
+    chunk = 1 << 20
+    for lo in range(0, flat.size, chunk):
+        d = np.abs(flat[lo:lo + chunk, None] - E2M1_GRID[None, :])
+        dmin = d.min(axis=1, keepdims=True)
+        is_min = d == dmin
+        n_min = is_min.sum(axis=1)
+        first = np.argmax(is_min, axis=1)            # lowest code at the minimum
+        # a tie is always between two adjacent codes; keep the even one
+        tie_pick = np.where(first % 2 == 0, first, first + 1)
+        mag[lo:lo + chunk] = np.where(n_min == 2, tie_pick, first).astype(np.uint8)
+    sign = np.signbit(v).reshape(-1).astype(np.uint8)
+    return (mag | (sign << 3)).reshape(v.shape)
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, dtype=np.uint8)
+    val = E2M1_GRID[c & 7]
+    return np.where(c & 8, -val, val)
+
+
+def quantize_mxfp4_rows(x: np.ndarray, ncols: Optional[int] = None):
+    """Quantize each row of x in consecutive 32-element blocks.
+
+    Only the first ``ncols`` columns are quantized (default: all); a last block
+    that is cut short is padded with zeros, which do not change its absmax.
+    Returns (codes uint8 [rows, nblocks*32], E int32 [rows, nblocks]); padded
+    positions hold code 0.
+    """
+    x = np.asarray(x, dtype=F32)
+    rows, cols = x.shape
+    n = cols if ncols is None else ncols
+    nb = -(-n // MX_BLOCK)
+    xp = np.zeros((rows, nb * MX_BLOCK), dtype=F32)
+    xp[:, :n] = x[:, :n]
+    blocks = xp.reshape(rows, nb, MX_BLOCK)
+    E = mx_scale_exponent(np.max(np.abs(blocks), axis=2))
+    # v = x * 2^-E is exact in float64 (and in float32)
+    v = blocks.astype(np.float64) * np.ldexp(1.0, -E.astype(np.int64))[:, :, None]
+    codes = e2m1_encode(v).reshape(rows, nb * MX_BLOCK)
+    return codes, E
+
+
+def mxfp4_dequant(codes: np.ndarray, E: np.ndarray) -> np.ndarray:
+    """Exact float64 value of row-blocked MXFP4 data: e2m1(code) * 2^E."""
+    rows, cols = codes.shape
+    nb = cols // MX_BLOCK
+    vals = e2m1_decode(codes).reshape(rows, nb, MX_BLOCK)
+    return (vals * np.ldexp(1.0, E.astype(np.int64))[:, :, None]).reshape(rows, cols)
+
+
+# ---------------------------------------------------------------------------
+# A3: static activation flattening  [notes, Stage 1; gist-zh 2.1; gist-pt 2.1]
+#     Y = X W = (X diag(s)^-1)(diag(s) W);  s_j = sqrt(max|X_j| / max|W_j|)
+# ---------------------------------------------------------------------------
+
+def calib_absmax(X: np.ndarray) -> np.ndarray:
+    """a_j = max_t |X[t, j]| over the calibration tokens."""
+    return np.max(np.abs(np.asarray(X, dtype=F32)), axis=0).astype(F32)
+
+
+def saf_scales(act_absmax: np.ndarray, W: np.ndarray) -> np.ndarray:
+    """s_j = sqrt(fp32(a_j / b_j)) with b_j = max_n |W[j, n]|; s_j = 1 if a_j or b_j is 0."""
+    a = np.asarray(act_absmax, dtype=F32)
+    b = np.max(np.abs(np.asarray(W, dtype=F32)), axis=1).astype(F32)
+    ok = (a > 0) & (b > 0)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        s = np.sqrt((a / b).astype(F32)).astype(F32)
+    return np.where(ok, s, F32(1.0)).astype(F32)
+
+
+# ---------------------------------------------------------------------------
+# A4: saliency ordering  [notes, Stage 2: W^ = P diag(s) W = [W_s; W_r]]
+# ---------------------------------------------------------------------------
+
+def saliency_permutation(s: np.ndarray) -> np.ndarray:
+    """perm[i] = original channel at permuted position i: s descending, ties by index."""
+    return np.argsort(-np.asarray(s, dtype=F32), kind="stable").astype(np.int32)
+
+
+def fold_weight(W: np.ndarray, s: np.ndarray, perm: np.ndarray, dtype=F32) -> np.ndarray:
+    """W^[i, n] = s[perm[i]] * W[perm[i], n] (one rounding in ``dtype``)."""
+    W = np.asarray(W, dtype=dtype)
+    s = np.asarray(s, dtype=dtype)
+    return (s[perm][:, None] * W[perm, :]).astype(dtype)
+
+
+def fold_activation(X: np.ndarray, s: np.ndarray, perm: np.ndarray, round_bf16: bool = True,
+                    dtype=F32) -> np.ndarray:
+    """X^[m, i] = X[m, perm[i]] / s[perm[i]]: the producer's folded output.
+
+    With the offline fold of [notes, Stage 3] the previous layer emits this
+    directly; it is stored in bf16 (round to nearest even).
+    """
+    X = np.asarray(X, dtype=dtype)
+    s = np.asarray(s, dtype=dtype)
+    xh = (X[:, perm] / s[perm][None, :]).astype(dtype)
+    return bf16_rne(xh) if round_bf16 else xh
+
+
+# ---------------------------------------------------------------------------
+# serq_prepare  [notes, Stage 1-3; gist-zh 2.2]
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class Prepared:
+    fmt: str
+    K: int
+    N: int
+    r: int
+    s: np.ndarray            # fp32 [K], original channel order
+    perm: np.ndarray         # int32 [K]
+    s_perm: np.ndarray       # fp32 [K], s[perm]
+    inv_s: np.ndarray        # fp32 [K], 1 / s[perm]
+    W_hat: np.ndarray        # fp32 [K, N]
+    qw: np.ndarray           # INT4: int8 [N, K]; MXFP4: uint8 codes [N, K]
+    sw: Optional[np.ndarray]  # INT4: fp32 [N]
+    Ew: Optional[np.ndarray]  # MXFP4: int32 [N, K/32]
+    R: np.ndarray            # fp32 [r, N]
+    qR: np.ndarray           # INT4: int8 [N, r]; MXFP4: uint8 codes [N, nbR*32]
+    sR: Optional[np.ndarray]  # INT4: fp32 [N]
+    ER: Optional[np.ndarray]  # MXFP4: int32 [N, nbR]
+
+    def deq_w(self) -> np.ndarray:
+        """Dequantized main weight, [N, K] float64."""
+        if self.fmt == "int4":
+            return self.qw.astype(np.float64) * self.sw.astype(np.float64)[:, None]
+        return mxfp4_dequant(self.qw, self.Ew)
+
+    def deq_R(self) -> np.ndarray:
+        """Dequantized residual, [N, r] float64."""
+        if self.fmt == "int4":
+            return self.qR.astype(np.float64) * self.sR.astype(np.float64)[:, None]
+        return mxfp4_dequant(self.qR, self.ER)[:, : self.r]
+
+
+def prepare(W: np.ndarray, r: int, fmt: str, act_absmax: Optional[np.ndarray] = None,
+            s: Optional[np.ndarray] = None, columns: Optional[np.ndarray] = None) -> Prepared:
+    """Offline SERQ preparation of one linear (W is K x N, Y = X W).
+
+    1. SAF scales s from calibration absmax (or given s)       [notes, Stage 1]
+    2. saliency permutation, s descending                       [notes, Stage 2]
+    3. W^ = P diag(s) W                                        [notes, Stage 2]
+    4. RTN quantization of W^: INT4 per output channel over K,
+       MXFP4 per 32 along K                                     [gist-zh 3 (RTN)]
+    5. R = W^_s - Q(W^_s) on the first r rows, with Q the main
+       weight quantization                                      [notes, Stage 2]
+    6. Q(R): 4-bit, INT4 per output channel, MXFP4 per 32 along r  [gist-zh 2.2]
+
+    ``columns`` restricts steps 3-6 to a subset of output channels (the
+    quantization of each output channel is independent of the others); s and
+    perm always use all of W.
+    """
+    assert fmt in ("int4", "mxfp4")
+    W = np.asarray(W, dtype=F32)
+    K, N = W.shape
+    assert 0 <= r <= K
+    if s is None:
+        s = saf_scales(act_absmax, W)
+    s = np.asarray(s, dtype=F32)
+    perm = saliency_permutation(s)
+    s_perm = s[perm]
+    inv_s = (F32(1.0) / s_perm).astype(F32)
+    Wc = W if columns is None else W[:, columns]
+    W_hat = fold_weight(Wc, s, perm)                       # [K, Nc] fp32
+    Wt = np.ascontiguousarray(W_hat.T)                     # [Nc, K]
+    if fmt == "int4":
+        qw, sw = quantize_int4(Wt, axis=1)                 # per output channel over K
+        deq_s = (qw[:, :r].astype(F32) * sw[:, None]).astype(F32)
+        R = (Wt[:, :r] - deq_s).astype(F32)                # [Nc, r]
+        if r > 0:
+            qR, sR = quantize_int4(R, axis=1)
+        else:
+            qR, sR = np.zeros((Wt.shape[0], 0), np.int8), np.zeros(Wt.shape[0], F32)
+        return Prepared(fmt, K, N, r, s, perm, s_perm, inv_s, W_hat, qw, sw, None,
+                        np.ascontiguousarray(R.T), qR, sR, None)
+    qw, Ew = quantize_mxfp4_rows(Wt)                       # blocks of 32 along K
+    if r > 0:
+        nb_r = -(-r // MX_BLOCK)
+        deq = (e2m1_decode(qw[:, : nb_r * MX_BLOCK]).reshape(-1, nb_r, MX_BLOCK)
+               * np.ldexp(1.0, Ew[:, :nb_r].astype(np.int64))[:, :, None]).reshape(Wt.shape[0], -1)
+        deq = deq[:, :r].astype(F32)                        # exact in fp32
+        R = (Wt[:, :r] - deq).astype(F32)
+        qR, ER = quantize_mxfp4_rows(R)
+    else:
+        R = np.zeros((Wt.shape[0], 0), F32)
+        qR, ER = np.zeros((Wt.shape[0], 0), np.uint8), np.zeros((Wt.shape[0], 0), np.int32)
+    return Prepared(fmt, K, N, r, s, perm, s_perm, inv_s, W_hat, qw, None, Ew,
+                    np.ascontiguousarray(R.T), qR, None, ER)
+
+
+# ---------------------------------------------------------------------------
+# serq_quant_act: per-token activation quantization + salient slice
+#   [notes, 基础量化 and 量化推理: X^_q and X~_{s,q}]
+# ---------------------------------------------------------------------------
+
+@dataclasses.dataclass
+class QuantAct:
+    fmt: str
+    r: int
+    qx: np.ndarray            # INT4: int8 [M, K]; MXFP4: uint8 codes [M, K]
+    sx: Optional[np.ndarray]  # INT4: fp32 [M]
+    Ex: Optional[np.ndarray]  # MXFP4: int32 [M, K/32]
+    qxs: np.ndarray           # INT4: int8 [M, r]; MXFP4: uint8 codes [M, nbr*32]
+    sxs: Optional[np.ndarray]  # INT4: fp32 [M]
+    Exs: Optional[np.ndarray]  # MXFP4: int32 [M, nbr]
+
+    def deq_x(self) -> np.ndarray:
+        if self.fmt == "int4":
+            return self.qx.astype(np.float64) * self.sx.astype(np.float64)[:, None]
+        return mxfp4_dequant(self.qx, self.Ex)
+
+    def deq_xs(self) -> np.ndarray:
+        if self.fmt == "int4":
+            return self.qxs.astype(np.float64) * self.sxs.astype(np.float64)[:, None]
+        return mxfp4_dequant(self.qxs, self.Exs)[:, : self.r]
+
+
+def quant_act(Xhat: np.ndarray, r: int, fmt: str) -> QuantAct:
+    """Quantize X^ per token and, under its own scale, the salient slice X^[:, :r]."""
+    X = np.asarray(Xhat, dtype=F32)
+    M, K = X.shape
+    if fmt == "int4":
+        qx, sx = quantize_int4(X, axis=1)
+        if r > 0:
+            qxs, sxs = quantize_int4(X[:, :r], axis=1)
+        else:
+            qxs, sxs = np.zeros((M, 0), np.int8), np.zeros(M, F32)
+        return QuantAct(fmt, r, qx, sx, None, qxs, sxs, None)
+    qx, Ex = quantize_mxfp4_rows(X)
+    if r > 0:
+        qxs, Exs = quantize_mxfp4_rows(X, ncols=r)
+    else:
+        qxs, Exs = np.zeros((M, 0), np.uint8), np.zeros((M, 0), np.int32)
+    return QuantAct(fmt, r, qx, None, Ex, qxs, None, Exs)
+
+
+# ---------------------------------------------------------------------------
+# serq_linear: Y ~= X^_q W^_q + X~_{s,q} Q(R)   [notes, 量化推理]
+# ---------------------------------------------------------------------------
+
+def _exact_int_matmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
+    """Integer matmul a[M,K] @ b[K,N] via float64 (exact: |partial sums| << 2^53)."""
+    assert a.shape[1] * 49 < 2 ** 52
+    c = np.asarray(a, dtype=np.float64) @ np.asarray(b, dtype=np.float64)
+    ci = c.astype(np.int64)
+    assert np.array_equal(ci, c)
+    return ci
+
+
+@dataclasses.dataclass
+class LinearOut:
+    Y: np.ndarray                      # float64 [M, N]
+    acc1: Optional[np.ndarray] = None  # INT4: int64 [M, N], sum_i qx * qw
+    acc2: Optional[np.ndarray] = None  # INT4: int64 [M, N], sum_{i<r} qxs * qR
+
+
+def linear(prep: Prepared, qa: QuantAct) -> LinearOut:
+    """Main 4-bit product plus the single residual product, no intermediate quantization."""
+    assert prep.fmt == qa.fmt and prep.r == qa.r
+    if prep.fmt == "int4":
+        acc1 = _exact_int_matmul(qa.qx, prep.qw.T)
+        acc2 = _exact_int_matmul(qa.qxs, prep.qR.T) if prep.r > 0 else np.zeros_like(acc1)
+        assert np.abs(acc1).max(initial=0) < 2 ** 31 and np.abs(acc2).max(initial=0) < 2 ** 31
+        Y = (acc1 * qa.sx.astype(np.float64)[:, None] * prep.sw.astype(np.float64)[None, :]
+             + acc2 * qa.sxs.astype(np.float64)[:, None] * prep.sR.astype(np.float64)[None, :])
+        return LinearOut(Y, acc1, acc2)
+    Y = qa.deq_x() @ prep.deq_w().T
+    if prep.r > 0:
+        Y = Y + qa.deq_xs() @ prep.deq_R().T
+    return LinearOut(Y)
+
+
+def serq_forward(X: np.ndarray, W: np.ndarray, r: int, fmt: str,
+                 X_calib: Optional[np.ndarray] = None):
+    """Whole pipeline on raw X (M x K) and W (K x N): calibrate, prepare, fold, quantize, multiply."""
+    a = calib_absmax(X if X_calib is None else X_calib)
+    prep = prepare(W, r, fmt, act_absmax=a)
+    Xh = fold_activation(X, prep.s, prep.perm)
+    qa = quant_act(Xh, r, fmt)
+    return prep, Xh, qa, linear(prep, qa)
+
+
+# ---------------------------------------------------------------------------
+# canonical packed byte layouts used for bit-exact comparisons
+# ---------------------------------------------------------------------------
+
+def pack_nibbles(codes: np.ndarray) -> np.ndarray:
+    """Two 4-bit codes per byte along the last axis: element 2j low nibble, 2j+1 high."""
+    c = (np.asarray(codes).astype(np.int16) & 0xF).astype(np.uint8)
+    if c.shape[-1] % 2:
+        c = np.concatenate([c, np.zeros(c.shape[:-1] + (1,), np.uint8)], axis=-1)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def e8m0(E: np.ndarray) -> np.ndarray:
+    """Biased E8M0 byte of a shared exponent."""
+    return (np.asarray(E, dtype=np.int32) + E8M0_BIAS).astype(np.uint8)
