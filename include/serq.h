@@ -1,0 +1,194 @@
+/*
+ * serq.h — C ABI of the SERQ W4A4 linear for NVIDIA B200 (sm_100a).
+ *
+ * SERQ ("Saliency-Aware Low-Rank Error Reconstruction for LLM Quantization",
+ * arXiv 2603.08185) runs a W4A4 linear layer as
+ *
+ *     Y ~= X^_q . W^_q  +  X~_{s,q} . Q(R)
+ *
+ * ("量化推理" formula of the dihengye.cn reading notes, Stage 2), where
+ *   - W^ = P . diag(s) . W is the weight after static activation flattening
+ *     (Stage 1, SAF) and the saliency row permutation P (Stage 2);
+ *   - R = W~_s - Q(W~_s) is the quantization error of the r salient rows of W^
+ *     (Stage 2, single-matrix compensation), itself quantized to 4 bits
+ *     (gist.science/zh summary, 2.2: "矩阵 R 本身也被量化为 4 位");
+ *   - X^ = X . diag(s)^-1 . P^T is produced directly by the previous layer,
+ *     into which 1/s and P are folded offline (Stage 3);
+ *   - X~_s = X^[:, :r] is the salient activation slice, quantized under its
+ *     own scale.
+ *
+ * Formats (gist.science/zh, 3: "INT4 或 MXFP4"):
+ *   SERQ_FMT_INT4  : symmetric INT4 codes in [-7, 7] (s = max|x| / 7, the
+ *                    "基础量化" formula with n = 4), fp32 scales: per token for
+ *                    activations, per output channel for W^ and R.
+ *   SERQ_FMT_MXFP4 : E2M1 codes with one E8M0 exponent per 32 consecutive
+ *                    elements along the reduction axis (OCP MX v1.0).
+ *
+ * Conventions
+ *   - Matrices are row-major. W is K x N (input channels x output channels,
+ *     the math layout of Y = X W). Activations are M x K (tokens x channels).
+ *   - 4-bit codes are packed two per byte along K: element 2j in the low
+ *     nibble, 2j+1 in the high nibble. INT4 codes are two's complement.
+ *     E2M1 codes are 0..15 (bit 3 = sign). E8M0 bytes are E + 127.
+ *   - MXFP4 scale bytes are stored in "atoms" of 128 rows x 4 blocks (512 B):
+ *     byte (row, block) of a tensor with nblk blocks per row lives at
+ *         ((row / 128) * ceil(nblk / 4) + block / 4) * 512
+ *           + (row % 32) * 16 + ((row % 128) / 32) * 4 + block % 4
+ *     which is the layout the tensor cores read scale factors in.
+ *   - The residual width is padded: rp = round_up(r, 64) (0 when r = 0).
+ *     Packed salient/residual rows have rp/2 bytes; codes past r are 0.
+ *   - All device pointers must be 16-byte aligned. Calls that take a
+ *     stream are asynchronous on it unless stated otherwise; pass NULL for
+ *     the legacy default stream.
+ *   - Errors are returned as serq_status; nothing aborts or throws across
+ *     the ABI. serq_last_error() gives a message for the calling thread.
+ *   - The library owns serq_weight and its device buffers; the caller owns
+ *     every other buffer.
+ */
+#ifndef SERQ_H
+#define SERQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* serq_stream; /* a cudaStream_t */
+
+typedef enum {
+    SERQ_OK = 0,
+    SERQ_EINVAL = 1,       /* bad argument: shape, pointer, alignment, format */
+    SERQ_EUNSUPPORTED = 2, /* device is not sm_100 or shape outside the kernels' range */
+    SERQ_ENOMEM = 3,       /* device allocation failed (serq_prepare only) */
+    SERQ_ECUDA = 4,        /* a CUDA runtime call failed */
+    SERQ_ETIMEOUT = 5      /* a kernel gave up waiting on a pipeline barrier */
+} serq_status;
+
+typedef enum { SERQ_FMT_INT4 = 0, SERQ_FMT_MXFP4 = 1 } serq_format;
+
+typedef struct serq_weight serq_weight; /* opaque prepared linear */
+
+/* ------------------------------------------------------------------------
+ * Calibration helper.
+ * Column absmax a_j = max_t |X[t, j]| of bf16 activations X (M x K, device),
+ * written to absmax (K floats, device). Feeds serq_prepare_desc.act_absmax
+ * (Stage 1: the SAF scales are set from calibration activations).
+ * Errors: EINVAL for M < 1, K < 1, NULL or unaligned pointers.
+ * ------------------------------------------------------------------------ */
+serq_status serq_calib_absmax(const void* X, int M, int K, float* absmax, serq_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Offline preparation (Stages 1-3 of the reading notes; gist.science/zh 2.1-2.3).
+ *
+ *   s_j  = sqrt(a_j / max_n |W[j, n]|)   (s_j = 1 if either is 0), unless s is given
+ *   perm = channels sorted by s descending (ties: lower index first)
+ *   W^   = P diag(s) W;  W^_q = RTN quantization of W^ (INT4 per output channel,
+ *          MXFP4 per 32 along K)
+ *   R    = W^[:r] - deq(W^_q)[:r];  Q(R) = INT4 per output channel / MXFP4 per 32 along r
+ *
+ * Inputs (device): W bf16 K x N; act_absmax fp32[K] or s fp32[K] (exactly one
+ * non-NULL). Requirements: K % 128 == 0, N % 128 == 0, 0 <= r <= K.
+ * On success *out owns device copies of perm, s, 1/s[perm], W^_q, Q(R) and
+ * their scales. Synchronizes the stream. Errors: EINVAL, EUNSUPPORTED,
+ * ENOMEM, ECUDA (nothing is leaked on failure).
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int K, N, r;
+    int fmt;                  /* serq_format */
+    const void* W;            /* device bf16 [K][N] */
+    const float* act_absmax;  /* device fp32 [K], or NULL when s is given */
+    const float* s;           /* device fp32 [K], or NULL */
+} serq_prepare_desc;
+
+serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_stream stream);
+void serq_weight_destroy(serq_weight* w);
+
+/* Device views of a prepared weight (all pointers owned by the weight).
+ *   perm   int32[K]   permuted position -> original channel
+ *   s      fp32[K]    SAF scales, original channel order
+ *   inv_s  fp32[K]    1 / s[perm[i]], permuted order (for the producer fold)
+ *   wq     u8[N][K/2]         packed W^_q, K-major
+ *   w_scale  INT4: fp32[N];   MXFP4: E8M0 atoms over (N rows, K/32 blocks)
+ *   rq     u8[N][rp/2]        packed Q(R), r-major
+ *   r_scale  INT4: fp32[N];   MXFP4: E8M0 atoms over (N rows, rp/32 blocks)   */
+typedef struct {
+    int K, N, r, rp, fmt;
+    const int32_t* perm;
+    const float* s;
+    const float* inv_s;
+    const uint8_t* wq;
+    size_t wq_bytes;
+    const void* w_scale;
+    size_t w_scale_bytes;
+    const uint8_t* rq;
+    size_t rq_bytes;
+    const void* r_scale;
+    size_t r_scale_bytes;
+} serq_weight_view;
+
+serq_status serq_weight_get_view(const serq_weight* w, serq_weight_view* out);
+
+/* ------------------------------------------------------------------------
+ * Producer fold (Stage 3: "行/列排列离线合并到权重中"; gist.science/zh 2.3).
+ * dst[row][i] = bf16(src[row][perm[i]] / s[perm[i]]) for a row-major bf16
+ * matrix whose K columns are this layer's input channels: the producer's
+ * weight (then X_prev . dst = X^), or an activation block (then dst = X^).
+ * src, dst: device, rows x K, must not overlap. Errors: EINVAL.
+ * ------------------------------------------------------------------------ */
+serq_status serq_fold_producer(const serq_weight* w, const void* src, int rows, void* dst,
+                               serq_stream stream);
+
+/* ------------------------------------------------------------------------
+ * Runtime activation quantization ("基础量化" per token; X~_{s,q} of "量化推理").
+ *
+ * Xhat: device bf16 [M][K]. Outputs (device, caller-allocated; sizes from
+ * serq_act_buffer_sizes):
+ *   INT4 : xq u8[M][K/2], xs fp32[M] (= max_i|x|/7), xsq u8[M][rp/2], xss fp32[M]
+ *          (= max_{i<r}|x|/7); codes rne(x / s) clipped to [-7, 7].
+ *   MXFP4: xq u8[M][K/2], xs E8M0 atoms (M rows, K/32 blocks), xsq u8[M][rp/2],
+ *          xss E8M0 atoms (M rows, rp/32 blocks; the slice's own blocks over
+ *          its first r columns, a short last block padded with zeros).
+ *   Scale bytes of atom rows >= M are not written.
+ * xsq/xss may be NULL when r == 0. Requirements: K % 128 == 0, 0 <= r <= K.
+ * Errors: EINVAL.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    size_t xq, xs, xsq, xss;
+} serq_act_sizes;
+
+serq_status serq_act_buffer_sizes(int M, int K, int r, int fmt, serq_act_sizes* out);
+serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void* xq, void* xs,
+                           void* xsq, void* xss, serq_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The SERQ linear (the "量化推理" formula): one kernel launch computing
+ *   MXFP4: Y = bf16( sum over K of X^_q W^_q  +  sum over r of X~_{s,q} Q(R) ),
+ *          both block-scaled products accumulated into one fp32 tile;
+ *   INT4 : acc1 = sum_i qx qw, acc2 = sum_{i<r} qxs qR (int32, exact),
+ *          Y = bf16(acc1 * xs[m] * w_scale[n] + acc2 * xss[m] * r_scale[n]).
+ * Inputs are serq_quant_act's outputs for the same (M, K, r, fmt).
+ * Y: device bf16 [M][N]. acc_dbg: NULL, or (INT4 only) device int32
+ * [2][M][N] receiving acc1 and acc2.
+ * Errors: EINVAL (shape/format mismatch with w, NULL/unaligned pointers),
+ * EUNSUPPORTED (not an sm_100 device).
+ * ------------------------------------------------------------------------ */
+serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void* xs,
+                        const void* xsq, const void* xss, void* Y, int32_t* acc_dbg,
+                        serq_stream stream);
+
+/* Synchronizes the stream, then reports (and clears) any device-side pipeline
+ * timeout recorded by this library's kernels on the current device:
+ * SERQ_ETIMEOUT if one occurred since the last call, else SERQ_OK
+ * (SERQ_ECUDA if the stream itself failed). */
+serq_status serq_device_status(serq_stream stream);
+
+const char* serq_last_error(void); /* thread-local message of the last failure */
+const char* serq_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SERQ_H */

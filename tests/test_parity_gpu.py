@@ -1,0 +1,92 @@
+"""GPU parity: every stage of the CUDA path against the CPU oracle.
+
+Bit-exact: calibration absmax, SAF scales, permutation, 1/s, folded
+activations, packed codes and scales of W^_q, Q(R), X^_q, X~_{s,q}, and the
+INT4 int32 accumulators. Within 2e-3 (max abs error over the row, divided by
+the row's L2 norm): the bf16 output Y.
+"""
+
+import numpy as np
+import pytest
+
+from oracle import serq_oracle as O
+from synth import activations, weights, workload
+
+from parity_util import compare_act, compare_weight, compare_y, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+def _check(X, W, r, fmt, X_calib=None):
+    res = run_gpu(X, W, r, fmt, X_calib=X_calib)
+    M, K = X.shape
+    a = O.calib_absmax(X if X_calib is None else X_calib)
+    assert np.array_equal(res["a"].view(np.uint32), a.view(np.uint32)), "calibration absmax"
+    prep = O.prepare(W, r, fmt, act_absmax=a)
+    compare_weight(res["view"], prep)
+    Xh = O.fold_activation(X, prep.s, prep.perm)
+    assert np.array_equal(res["Xh"].view(np.uint32), Xh.view(np.uint32)), "folded activations"
+    qa = O.quant_act(Xh, r, fmt)
+    compare_act(res, qa, M, K, r)
+    out = O.linear(prep, qa)
+    if fmt == "int4":
+        assert np.array_equal(res["acc"][0], out.acc1), "acc1"
+        assert np.array_equal(res["acc"][1], out.acc2), "acc2"
+    return compare_y(res["Y"], out.Y)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_tiny_workload(fmt):
+    wl = workload("tiny_int4")
+    lin = wl.linears[0]
+    _check(lin.X(wl.M), lin.W(), lin.r, fmt)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("M,K,N,r", [
+    (1, 256, 256, 16),        # a single token
+    (77, 384, 384, 32),       # ragged M, K % 256 == 128 (half K-tile), N % 256 == 128 (half N-tile)
+    (200, 512, 640, 0),       # r = 0: plain W4A4
+    (130, 1024, 512, 128),    # two M tiles, the pages' rank
+    (64, 512, 256, 256),      # r = 256
+    (129, 768, 1280, 40),     # r not a multiple of 32 (short salient block)
+    (33, 256, 256, 256),      # r = K
+])
+def test_shapes(fmt, M, K, N, r):
+    X = activations(1000 + M, M, K, max(1, K // 100), "lognormal", 50.0)
+    W = weights(2000 + K, K, N)
+    _check(X, W, r, fmt)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_degenerate_rows(fmt):
+    # a zero row, an all-equal row, a row with one huge outlier, exact ties
+    M, K, N, r = 8, 256, 256, 16
+    X = activations(7, M, K, 3, "const", 30.0)
+    X[1] = 0.0
+    X[2] = 1.5
+    X[3] = 0.0
+    X[3, 100] = 1000.0
+    X[4, :] = np.where(np.arange(K) % 2 == 0, 3.5, -3.5)
+    W = weights(8, K, N)
+    W[5] = 0.0  # a zero weight row -> s_j = 1
+    _check(X, W, r, fmt, X_calib=X)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_calibration_on_separate_draw(fmt):
+    M, K, N, r = 16, 512, 256, 128
+    X = activations(21, M, K, 5, "const", 50.0)
+    Xc = activations(22, 300, K, 5, "const", 50.0)
+    W = weights(23, K, N)
+    _check(X, W, r, fmt, X_calib=Xc)
+
+
+def test_residual_reduces_error_on_gpu():
+    # same trend as the oracle: the salient correction lowers the layer error
+    wl = workload("tiny_int4")
+    lin = wl.linears[0]
+    X, W = lin.X(wl.M), lin.W()
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    errs = [np.linalg.norm(run_gpu(X, W, r, "int4")["Y"] - ref) for r in (0, 16, 64)]
+    assert errs[1] < errs[0] and errs[2] < errs[1]

@@ -1,0 +1,23 @@
+"""SERQ W4A4 linear for NVIDIA B200 (sm_100a): Python binding of libserq.so.
+
+Y ~= X^_q W^_q + X~_{s,q} Q(R) -- saliency-aware single-matrix low-rank error
+reconstruction ("SERQ: Saliency-Aware Low-Rank Error Reconstruction for LLM
+Quantization"). The computation runs in the CUDA kernels of libserq.so;
+this package only marshals arguments (see include/serq.h).
+"""
+
+from .serq import (  # noqa: F401
+    QuantAct,
+    SerqWeight,
+    alloc_act,
+    serq_act_buffer_sizes,
+    serq_calib_absmax,
+    serq_device_status,
+    serq_fold_producer,
+    serq_linear,
+    serq_prepare,
+    serq_quant_act,
+    serq_version,
+    serq_weight_get_view,
+)
+from ._native import SerqError  # noqa: F401

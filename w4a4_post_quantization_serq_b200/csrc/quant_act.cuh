@@ -1,0 +1,211 @@
+// serq_quant_act kernels: per-token activation quantization and the salient
+// slice X~_s = X^[:, :r] under its own scale.
+//
+// INT4  ("基础量化", reading notes): s = max|x| / 7, q = clip(rne(x / s), -7, 7),
+//       one fp32 scale per token; the slice uses the absmax of its r columns.
+// MXFP4 (OCP MX v1.0, named by the pages as MXFP4): per 32-element block,
+//       E = floor(log2 amax) - 2 (clamped to [-127, 127]), codes = E2M1
+//       round-to-nearest-even of x * 2^-E (saturating at 6).
+//
+// Every quantization decision is made in IEEE fp32 with one rounding per
+// operation (explicit __fdiv_rn; no contraction), so the codes match a
+// scalar fp32 restatement bit for bit.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace serq {
+
+constexpr int kQuantThreads = 256;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        f[2 * i] = __uint_as_float(w[i] << 16);
+        f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+}
+
+// INT4 code of x under scale s (two's complement nibble); 0 when s == 0.
+__device__ __forceinline__ uint32_t int4_code(float x, float s) {
+    if (!(s > 0.0f)) return 0u;
+    float q = rintf(__fdiv_rn(x, s));
+    q = fminf(fmaxf(q, -7.0f), 7.0f);
+    return static_cast<uint32_t>(static_cast<int>(q)) & 0xFu;
+}
+
+// Shared MX exponent of a block from its absmax: floor(log2 amax) - 2, read
+// off the fp32 exponent field; zero and subnormal maxima give -127.
+__device__ __forceinline__ int mx_exponent(float amax) {
+    const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFFu);
+    if (e == 0) return -127;
+    const int E = e - 127 - 2;
+    return E < -127 ? -127 : E;
+}
+
+// 2^-E for E in [-127, 125] (always a normal float).
+__device__ __forceinline__ float mx_inv_scale(int E) {
+    return __uint_as_float(static_cast<uint32_t>(127 - E) << 23);
+}
+
+// Eight already-scaled floats -> eight E2M1 codes packed in a 32-bit word,
+// element 0 in the lowest nibble (round to nearest even, saturate to +-6).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&v)[8]) {
+    uint32_t r;
+    asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+        "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+        "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+        : "=r"(r)
+        : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+    return r;
+}
+
+// Byte offset of the scale of (row, block) in the tensor-core scale atom
+// layout: 128 rows x 4 blocks per 512-byte atom, atoms ordered by row block
+// then block group.
+__device__ __forceinline__ size_t sf_atom_offset(int row, int blk, int atoms_per_rowblock) {
+    return (static_cast<size_t>(row >> 7) * atoms_per_rowblock + (blk >> 2)) * 512u +
+           static_cast<size_t>((row & 31) * 16 + ((row >> 5) & 3) * 4 + (blk & 3));
+}
+
+__device__ __forceinline__ float block_max2(float& a, float& b, float* red) {
+    // reduce two maxima over the CTA; red holds 2 * (kQuantThreads / 32) floats
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, o));
+        b = fmaxf(b, __shfl_xor_sync(0xFFFFFFFFu, b, o));
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane == 0) {
+        red[warp] = a;
+        red[32 + warp] = b;
+    }
+    __syncthreads();
+    a = red[0];
+    b = red[32];
+#pragma unroll
+    for (int w = 1; w < kQuantThreads / 32; ++w) {
+        a = fmaxf(a, red[w]);
+        b = fmaxf(b, red[32 + w]);
+    }
+    return a;
+}
+
+// One CTA per token row. MAXC = 16-byte chunks held per thread (K <= 8 * 256 * MAXC).
+template <int MAXC>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
+                      float* __restrict__ xs, uint32_t* __restrict__ xsq, float* __restrict__ xss) {
+    __shared__ float red[64];
+    const int m = blockIdx.x;
+    const int nchunk = K >> 3;
+    const uint4* row = X + static_cast<size_t>(m) * nchunk;
+    uint4 v[MAXC];
+    float amax = 0.0f, amax_s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = threadIdx.x + j * kQuantThreads;
+        if (c < nchunk) {
+            v[j] = __ldg(row + c);
+            float f[8];
+            bf16x8_to_f32(v[j], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float a = fabsf(f[e]);
+                amax = fmaxf(amax, a);
+                if (c * 8 + e < r) amax_s = fmaxf(amax_s, a);
+            }
+        }
+    }
+    block_max2(amax, amax_s, red);
+    const float s = __fdiv_rn(amax, 7.0f);
+    const float ss = __fdiv_rn(amax_s, 7.0f);
+    if (threadIdx.x == 0) {
+        xs[m] = s;
+        if (rp > 0) xss[m] = ss;
+    }
+    const int nchunk_s = rp >> 3;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = threadIdx.x + j * kQuantThreads;
+        if (c < nchunk) {
+            float f[8];
+            bf16x8_to_f32(v[j], f);
+            uint32_t w = 0;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) w |= int4_code(f[e], s) << (4 * e);
+            xq[static_cast<size_t>(m) * nchunk + c] = w;
+            if (c < nchunk_s) {
+                uint32_t ws = 0;
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (c * 8 + e < r) ws |= int4_code(f[e], ss) << (4 * e);
+                xsq[static_cast<size_t>(m) * nchunk_s + c] = ws;
+            }
+        }
+    }
+}
+
+// One CTA per token row; four consecutive threads share one 32-element block.
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
+                       uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
+                       uint8_t* __restrict__ xss_atoms) {
+    const int m = blockIdx.x;
+    const int nchunk = K >> 3;
+    const int atoms_k = (K / 32 + 3) / 4;
+    const int nchunk_s = rp >> 3;
+    const int atoms_s = (rp / 32 + 3) / 4;
+    const uint4* row = X + static_cast<size_t>(m) * nchunk;
+    const int iters = (nchunk + kQuantThreads - 1) / kQuantThreads;
+    for (int j = 0; j < iters; ++j) {
+        const int c = threadIdx.x + j * kQuantThreads;
+        const bool valid = c < nchunk;
+        float f[8];
+        if (valid) {
+            bf16x8_to_f32(__ldg(row + c), f);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) f[e] = 0.0f;
+        }
+        float a = 0.0f, as = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            a = fmaxf(a, fabsf(f[e]));
+            if (c * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
+        }
+        // the four chunks of a block sit in four consecutive lanes
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+        as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+        as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+        if (!valid) continue;
+        const int blk = c >> 2;
+        const int E = mx_exponent(a);
+        const float inv = mx_inv_scale(E);
+        float g[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
+        xq[static_cast<size_t>(m) * nchunk + c] = e2m1x8(g);
+        if ((threadIdx.x & 3) == 0) xs_atoms[sf_atom_offset(m, blk, atoms_k)] = static_cast<uint8_t>(E + 127);
+        if (c < nchunk_s) {
+            // the slice's own block over its first r columns (zeros beyond r)
+            const int Es = mx_exponent(as);
+            const float invs = mx_inv_scale(Es);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = (c * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+            xsq[static_cast<size_t>(m) * nchunk_s + c] = e2m1x8(g);
+            if ((threadIdx.x & 3) == 0)
+                xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
+        }
+    }
+}
+
+}  // namespace serq

@@ -1,0 +1,173 @@
+"""Python binding of the SERQ C ABI: same names as include/serq.h.
+
+Argument marshalling only. Device buffers are torch CUDA tensors, the stream
+is torch's current stream, and every computation runs in libserq.so's CUDA
+kernels. There is no CPU path: calls fail when the library is not built or
+no sm_100 device is present.
+"""
+
+from __future__ import annotations
+
+import ctypes
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import torch
+
+from . import _native as N
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t: Optional[torch.Tensor]) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda or not t.is_contiguous():
+        raise ValueError("expected a contiguous CUDA tensor")
+    return t.data_ptr()
+
+
+def _fmt(fmt) -> int:
+    return N.FMT[fmt] if isinstance(fmt, str) else int(fmt)
+
+
+class _DeviceView:
+    """Zero-copy torch view of library-owned device memory."""
+
+    def __init__(self, ptr: int, shape, typestr: str, owner):
+        self.owner = owner
+        self.__cuda_array_interface__ = {"shape": tuple(shape), "typestr": typestr, "data": (ptr, False),
+                                         "version": 3, "strides": None}
+
+
+def _view(ptr, shape, typestr, owner) -> torch.Tensor:
+    return torch.as_tensor(_DeviceView(ptr, shape, typestr, owner), device="cuda")
+
+
+class SerqWeight:
+    """A prepared SERQ linear (owns its device buffers through the library)."""
+
+    def __init__(self, handle: int, K: int, N_: int, r: int, fmt: int):
+        self.handle = ctypes.c_void_p(handle)
+        self.K, self.N, self.r, self.fmt = K, N_, r, fmt
+        self.rp = ((r + 63) // 64) * 64 if r > 0 else 0
+
+    def __del__(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            N.load().serq_weight_destroy(self.handle)
+            self.handle = None
+
+    def view(self) -> Dict[str, torch.Tensor]:
+        """Device tensors of perm, s, inv_s, packed W^_q / Q(R) and their scales."""
+        return serq_weight_get_view(self)
+
+
+def serq_calib_absmax(X: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    M, K = X.shape
+    if out is None:
+        out = torch.empty(K, dtype=torch.float32, device=X.device)
+    N.check(N.load().serq_calib_absmax(_ptr(X), M, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def serq_prepare(W: torch.Tensor, r: int, fmt, act_absmax: Optional[torch.Tensor] = None,
+                 s: Optional[torch.Tensor] = None, stream=None) -> SerqWeight:
+    """Offline preparation of one linear; W is bf16 K x N (Y = X W). Synchronizes."""
+    if W.dtype != torch.bfloat16:
+        raise ValueError("W must be bfloat16")
+    K, N_ = W.shape
+    desc = N.PrepareDesc(K, N_, r, _fmt(fmt), _ptr(W), _ptr(act_absmax), _ptr(s))
+    h = ctypes.c_void_p()
+    N.check(N.load().serq_prepare(ctypes.byref(desc), ctypes.byref(h), _stream(stream)))
+    return SerqWeight(h.value, K, N_, r, _fmt(fmt))
+
+
+def serq_weight_get_view(w: SerqWeight) -> Dict[str, torch.Tensor]:
+    v = N.WeightView()
+    N.check(N.load().serq_weight_get_view(w.handle, ctypes.byref(v)))
+    out = {
+        "perm": _view(v.perm, (v.K,), "<i4", w),
+        "s": _view(v.s, (v.K,), "<f4", w),
+        "inv_s": _view(v.inv_s, (v.K,), "<f4", w),
+        "wq": _view(v.wq, (v.N, v.K // 2), "|u1", w),
+    }
+    if v.fmt == 0:
+        out["w_scale"] = _view(v.w_scale, (v.N,), "<f4", w)
+        if v.rp > 0:
+            out["rq"] = _view(v.rq, (v.N, v.rp // 2), "|u1", w)
+            out["r_scale"] = _view(v.r_scale, (v.N,), "<f4", w)
+    else:
+        out["w_scale"] = _view(v.w_scale, (v.w_scale_bytes,), "|u1", w)
+        if v.rp > 0:
+            out["rq"] = _view(v.rq, (v.N, v.rp // 2), "|u1", w)
+            out["r_scale"] = _view(v.r_scale, (v.r_scale_bytes,), "|u1", w)
+    return out
+
+
+def serq_fold_producer(w: SerqWeight, src: torch.Tensor, dst: Optional[torch.Tensor] = None,
+                       stream=None) -> torch.Tensor:
+    """dst[row, i] = bf16(src[row, perm[i]] / s[perm[i]])."""
+    rows = src.shape[0]
+    if dst is None:
+        dst = torch.empty_like(src)
+    N.check(N.load().serq_fold_producer(w.handle, _ptr(src), rows, _ptr(dst), _stream(stream)))
+    return dst
+
+
+def serq_act_buffer_sizes(M: int, K: int, r: int, fmt) -> Dict[str, int]:
+    sz = N.ActSizes()
+    N.check(N.load().serq_act_buffer_sizes(M, K, r, _fmt(fmt), ctypes.byref(sz)))
+    return {"xq": sz.xq, "xs": sz.xs, "xsq": sz.xsq, "xss": sz.xss}
+
+
+@dataclass
+class QuantAct:
+    M: int
+    K: int
+    r: int
+    fmt: int
+    xq: torch.Tensor
+    xs: torch.Tensor
+    xsq: Optional[torch.Tensor]
+    xss: Optional[torch.Tensor]
+
+
+def alloc_act(M: int, K: int, r: int, fmt, device="cuda") -> QuantAct:
+    sz = serq_act_buffer_sizes(M, K, r, fmt)
+
+    def buf(n):
+        return torch.empty(max(n, 16), dtype=torch.uint8, device=device) if n > 0 else None
+    return QuantAct(M, K, r, _fmt(fmt), buf(sz["xq"]), buf(sz["xs"]), buf(sz["xsq"]), buf(sz["xss"]))
+
+
+def serq_quant_act(Xhat: torch.Tensor, r: int, fmt, out: Optional[QuantAct] = None, stream=None) -> QuantAct:
+    """Per-token INT4 / MXFP4 quantization of X^ and of its salient slice X^[:, :r]."""
+    M, K = Xhat.shape
+    if out is None:
+        out = alloc_act(M, K, r, fmt, Xhat.device)
+    N.check(N.load().serq_quant_act(_ptr(Xhat), M, K, r, _fmt(fmt), _ptr(out.xq), _ptr(out.xs), _ptr(out.xsq),
+                                    _ptr(out.xss), _stream(stream)))
+    return out
+
+
+def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
+                acc_dbg: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Y = X^_q W^_q + X~_{s,q} Q(R), bf16 M x N, in one kernel launch."""
+    if Y is None:
+        Y = torch.empty(qa.M, w.N, dtype=torch.bfloat16, device=qa.xq.device)
+    N.check(N.load().serq_linear(w.handle, qa.M, _ptr(qa.xq), _ptr(qa.xs), _ptr(qa.xsq), _ptr(qa.xss), _ptr(Y),
+                                 _ptr(acc_dbg), _stream(stream)))
+    return Y
+
+
+def serq_device_status(stream=None) -> None:
+    """Synchronize and raise SerqError(SERQ_ETIMEOUT) if a kernel wait timed out."""
+    N.check(N.load().serq_device_status(_stream(stream)))
+
+
+def serq_version() -> str:
+    return N.load().serq_version().decode()
