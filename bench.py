@@ -1,0 +1,433 @@
+#!/usr/bin/env python
+"""Benchmark of the SERQ W4A4 linear on B200; prints one JSON line.
+
+One step = the whole hot path over one batch of the LLaMA-3-8B-shaped MLP
+workload at M = 2048 tokens, r = 128, MXFP4:
+    serq_quant_act(X^_gu) -> serq_linear(gate|up, N = 2 x 14336)
+    serq_quant_act(X^_dn) -> serq_linear(down, K = 14336)
+value = sum over the step of 2*M*N*(K+r) / device time (TOPS), max over ranks.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+--impl reference times the CPU oracle (the only other implementation of the
+method here) on a bounded row sample of the same workload.
+Multi-GPU runs are independent replicas (the linear has no exchange step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "serq_linear TOPS (2·M·N·(K+r)/t) and % of FP4 peak; decode GB/s; overhead vs r=0"
+WORKLOAD = "mlp_mxfp4"
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+CAPTURED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-rows", type=int, default=64, help="token rows of the oracle's timed sample")
+    ap.add_argument("--no-extras", action="store_true", help="skip the r=0, INT4 and e2e side measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (for profiler runs)")
+    ap.add_argument("--only", default=None, help="time only the named linear of the workload (profiling)")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------- distributed
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        backend = "nccl" if _cuda_ok() else "gloo"
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return world, rank, local, pg
+
+
+def _cuda_ok():
+    import torch
+    return torch.cuda.is_available()
+
+
+def barrier(pg):
+    if pg is not None:
+        import torch
+        if torch.cuda.is_available():
+            pg.barrier(device_ids=[torch.cuda.current_device()])
+        else:
+            pg.barrier()
+
+
+def max_over_ranks(pg, value: float) -> float:
+    if pg is None:
+        return value
+    import torch
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """NVML samples (every 10 ms) of the SM clock, power and clock-event reasons.
+
+    Read-only queries; sampling runs in a thread from start() to stop().
+    """
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device_index: int):
+        import threading
+        self.samples = []
+        self.window = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            self.nv = nv
+            self.h = nv.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self.h, nv.NVML_CLOCK_SM)
+        except Exception:  # no NVML: no clock record
+            self.nv = None
+            return
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append((time.perf_counter(), nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM),
+                                     nv.nvmlDeviceGetCurrentClocksEventReasons(self.h),
+                                     nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
+            except Exception:
+                pass
+            time.sleep(0.01)
+
+    def mark(self, t0, t1):
+        self.window = (t0, t1)
+
+    def stop(self):
+        if self._thread is None:
+            return None
+        self._stop.set()
+        self._thread.join(timeout=2)
+        if not self.samples:
+            return None
+        nv = self.nv
+        reasons = set()
+        for _, _, mask, _ in self.samples:
+            for name, attr in self.REASONS:
+                if hasattr(nv, attr) and mask & getattr(nv, attr):
+                    reasons.add(name)
+        inside = [s for s in self.samples if self.window and self.window[0] <= s[0] <= self.window[1]]
+        return {"sm_mhz": statistics.median(s[1] for s in self.samples), "sm_max_mhz": self.max_mhz,
+                "power_w_max": max(s[3] for s in self.samples), "samples": len(self.samples),
+                "samples_in_timed_region": len(inside),
+                "sm_mhz_timed_region": statistics.median(s[1] for s in inside) if inside else None,
+                "reasons": sorted(reasons), "source": "NVML, 10 ms period, 0.5 s pre-roll + timed region"}
+
+
+# ----------------------------------------------------------------- workload
+def linear_flops(M, lin):
+    return 2.0 * M * lin.N * (lin.K + lin.r)
+
+
+def build_layers(wl, r_override=None, device="cuda"):
+    """Device-resident inputs of the step: prepared weights, folded activations, buffers."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    layers = []
+    for lin in wl.linears:
+        r = lin.r if r_override is None else r_override
+        X = torch.from_numpy(lin.X(wl.M)).to(torch.bfloat16).to(device)
+        W = torch.from_numpy(lin.W()).to(torch.bfloat16).to(device)
+        a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(wl.M)).to(torch.bfloat16).to(device))
+        w = S.serq_prepare(W, r, lin.fmt, act_absmax=a)
+        Xh = S.serq_fold_producer(w, X)
+        del W, X
+        layers.append({"lin": lin, "r": r, "w": w, "Xh": Xh, "qa": S.alloc_act(wl.M, lin.K, r, lin.fmt, device),
+                       "Y": torch.empty(wl.M, lin.N, dtype=torch.bfloat16, device=device),
+                       "flops": 2.0 * wl.M * lin.N * (lin.K + r)})
+    torch.cuda.synchronize()
+    return layers
+
+
+def run_step(layers, gemm_events=None):
+    import w4a4_post_quantization_serq_b200 as S
+    for i, L in enumerate(layers):
+        S.serq_quant_act(L["Xh"], L["r"], L["lin"].fmt, out=L["qa"])
+        if gemm_events is not None:
+            gemm_events[i][0].record()
+        S.serq_linear(L["w"], L["qa"], Y=L["Y"])
+        if gemm_events is not None:
+            gemm_events[i][1].record()
+
+
+def time_steps(layers, steps, warmup, pg, per_gemm=True, sampler=None):
+    """Device time of `steps` steps (CUDA events on the launching stream)."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    for _ in range(warmup):
+        run_step(layers)
+    S.serq_device_status()
+    if sampler is not None:
+        # untimed pre-roll under the same load so the clock record has samples
+        t_end = time.perf_counter() + 0.5
+        while time.perf_counter() < t_end:
+            run_step(layers)
+            torch.cuda.synchronize()
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    start.record()
+    for k in range(steps):
+        run_step(layers, ev[k] if per_gemm else None)
+    end.record()
+    torch.cuda.synchronize()
+    if sampler is not None:
+        sampler.mark(t0, time.perf_counter())
+    barrier(pg)
+    S.serq_device_status()
+    total_ms = start.elapsed_time(end)
+    gemm_ms = [sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(steps)) / steps
+               for i in range(len(layers))] if per_gemm else None
+    return total_ms, gemm_ms
+
+
+def time_e2e(layers, steps, warmup):
+    """Same step through the public API with host buffers: pinned H2D of X^, D2H of Y, every step."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    host_in = [L["Xh"].cpu().pin_memory() for L in layers]
+    host_out = [torch.empty(L["Y"].shape, dtype=L["Y"].dtype).pin_memory() for L in layers]
+
+    def step():
+        for L, hi, ho in zip(layers, host_in, host_out):
+            L["Xh"].copy_(hi, non_blocking=True)
+            S.serq_quant_act(L["Xh"], L["r"], L["lin"].fmt, out=L["qa"])
+            S.serq_linear(L["w"], L["qa"], Y=L["Y"])
+            ho.copy_(L["Y"], non_blocking=True)
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    S.serq_device_status()
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+    return start.elapsed_time(end) / steps, h2d, d2h
+
+
+# ----------------------------------------------------------------- CPU oracle
+def cpu_oracle_prepare(wl, r_override=None):
+    """The oracle's offline preparation of every linear (not timed)."""
+    from oracle import serq_oracle as O
+    out = []
+    for lin in wl.linears:
+        r = lin.r if r_override is None else r_override
+        prep = O.prepare(lin.W(), r, lin.fmt, act_absmax=O.calib_absmax(lin.X_calib(wl.M)))
+        out.append((lin, r, prep, lin.X(wl.M)))
+    return out
+
+
+def cpu_oracle_step(prepared, rows):
+    """One timed oracle step on `rows` tokens: activation quantization + linear.
+
+    Returns (seconds, flops, cores)."""
+    from threadpoolctl import threadpool_info
+
+    from oracle import serq_oracle as O
+    t_total, flops = 0.0, 0.0
+    for lin, r, prep, X in prepared:
+        Xh = O.fold_activation(X[:rows], prep.s, prep.perm)
+        t0 = time.perf_counter()
+        qa = O.quant_act(Xh, r, lin.fmt)
+        O.linear(prep, qa)
+        t_total += time.perf_counter() - t0
+        flops += 2.0 * rows * lin.N * (lin.K + r)
+    cores = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    return t_total, flops, cores
+
+
+# ----------------------------------------------------------------- main
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def captured_traffic():
+    """DRAM bytes per launch from the committed ncu capture, or None once the
+    kernel source differs from the one the counters were taken on."""
+    import hashlib
+    try:
+        rec = json.load(open(CAPTURED_TRAFFIC_FILE))
+        src = os.path.join(ROOT, "w4a4_post_quantization_serq_b200", "csrc", "gemm_mxfp4.cuh")
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except (OSError, ValueError):
+        return None
+    return rec.get("dram_bytes_per_launch") if rec.get("source_sha256_prefix") == sha else None
+
+
+def reference_main(args, world, rank, pg):
+    """The CPU oracle on a bounded token sample of the same workload (rank 0 only)."""
+    from synth import workload
+    if rank != 0:
+        return
+    wl = workload(WORKLOAD)
+    rows = args.cpu_rows
+    prepared = cpu_oracle_prepare(wl)
+    for _ in range(args.warmup):
+        cpu_oracle_step(prepared, rows)
+    secs, flops, cores = [], 0.0, 1
+    t_start = time.perf_counter()
+    for _ in range(max(1, args.steps)):
+        t, flops, cores = cpu_oracle_step(prepared, rows)
+        secs.append(t)
+        if time.perf_counter() - t_start > 150:  # keep the run to a few minutes
+            break
+    mean_t = sum(secs) / len(secs)
+    tops = flops / mean_t / 1e12
+    sample = (f"{rows} of {wl.M} tokens of every linear ({', '.join(l.name for l in wl.linears)}), r=128: "
+              f"oracle quant_act + linear per step; offline prepare untimed")
+    line = {"impl": "reference", "metric": METRIC, "value": tops, "unit": "TOPS", "n_gpus": world,
+            "steps": len(secs), "warmup": args.warmup, "ms_per_step": mean_t * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64 (fp32 quantization decisions)",
+            "data": "synthetic", "config": {"workload": wl.description, "M_sampled": rows},
+            "cpu_baseline": {"value": tops, "unit": "TOPS", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": tops, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    world, rank, local, pg = dist_setup(args.gpus)
+    if args.impl == "reference":
+        reference_main(args, world, rank, pg)
+        if pg is not None:
+            pg.destroy_process_group()
+        return
+
+    import torch
+    import w4a4_post_quantization_serq_b200 as S  # noqa: F401  (fails loudly without libserq.so)
+    from synth import workload
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    wl = workload(WORKLOAD)
+    if args.only:
+        wl.linears = [l for l in wl.linears if l.name == args.only]
+        if not wl.linears:
+            raise SystemExit(f"no linear named {args.only}")
+    layers = build_layers(wl)
+    step_flops = sum(L["flops"] for L in layers)
+
+    sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
+    total_ms, gemm_ms = time_steps(layers, args.steps, args.warmup, pg, sampler=sampler)
+    clocks = sampler.stop() if sampler is not None else None
+    total_ms = max_over_ranks(pg, total_ms)
+    ms_per_step = total_ms / args.steps
+    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+    # dominant kernel: serq_linear_mxfp4_kernel; its largest launch (gate/up,
+    # two thirds of the step's flops) is the roofline's unit
+    peaks, peak_src = measured_peaks()
+    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    dom = max(range(len(layers)), key=lambda i: layers[i]["flops"])
+    achieved = layers[dom]["flops"] / (gemm_ms[dom] * 1e-3) / 1e12
+    traffic = captured_traffic()
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak, "traffic": traffic,
+                "kernel": "serq_linear_mxfp4_kernel", "launch": layers[dom]["lin"].name,
+                "flops_per_launch": layers[dom]["flops"],
+                "peak_source": f"{peak_src} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
+                               f"{FP4_OVER_BF16:g} (nominal dense FP4/BF16 ratio)",
+                "per_launch_us": {L["lin"].name: round(t * 1e3, 2) for L, t in zip(layers, gemm_ms)},
+                "all_launches_tflops": sum(L["flops"] for L in layers) / (sum(gemm_ms) * 1e-3) / 1e12,
+                "gemm_share_of_step": sum(gemm_ms) / ms_per_step}
+
+    line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e2m1, e8m0 per 32, fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": wl.description, "M": wl.M, "r": 128,
+                       "linears": [{"name": L["lin"].name, "K": L["lin"].K, "N": L["lin"].N} for L in layers],
+                       "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (a step touches ~300 MB)"},
+            "roofline": roofline, "gpu_launches": 2 * len(layers) * args.steps, "clocks": clocks}
+
+    if not args.no_extras and rank == 0:
+        # SERQ overhead: the same step with r = 0 (plain W4A4)
+        del layers
+        torch.cuda.empty_cache()
+        layers0 = build_layers(wl, r_override=0)
+        t0, g0 = time_steps(layers0, args.steps, args.warmup, None)
+        del layers0
+        torch.cuda.empty_cache()
+        line["overhead_vs_r0"] = {"ms_per_step_r0": t0 / args.steps, "step": ms_per_step / (t0 / args.steps) - 1,
+                                  "serq_linear": sum(gemm_ms) / sum(g0) - 1}
+        # end to end through the public API with host buffers
+        layers = build_layers(wl)
+        e2e_ms, h2d, d2h = time_e2e(layers, max(3, args.steps // 4), 2)
+        line["e2e"] = {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        del layers
+        torch.cuda.empty_cache()
+        # INT4: LLaMA-2-7B q_proj shape
+        wl2 = workload("qproj_int4")
+        layers2 = build_layers(wl2)
+        t2, g2 = time_steps(layers2, args.steps, args.warmup, None)
+        f2 = sum(L["flops"] for L in layers2)
+        line["int4_qproj"] = {"TOPS": f2 / (t2 / args.steps * 1e-3) / 1e12, "ms_per_step": t2 / args.steps,
+                              "serq_linear_us": g2[0] * 1e3,
+                              "frac_of_int8_peak": f2 / (g2[0] * 1e-3) / 1e12 / (peaks["bf16_tflops_sustained"] * 2)}
+        del layers2
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        secs, flops, cores = cpu_oracle_step(cpu_oracle_prepare(wl), args.cpu_rows)
+        line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+                                "sample": f"{args.cpu_rows} of {wl.M} tokens of every linear, oracle quant_act + "
+                                          f"linear ({secs:.1f} s); offline prepare untimed"}
+    if "e2e" not in line:
+        line["e2e"] = None
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
