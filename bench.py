@@ -250,6 +250,62 @@ def time_e2e(layers, steps, warmup):
     return start.elapsed_time(end) / steps, h2d, d2h
 
 
+def bench_decode(reps: int = 10, tokens=(1, 4, 16)):
+    """HBM-bound small-M serq_linear on the LLaMA-3-8B decode shapes.
+
+    For each shape, a pool of independently prepared copies of the weight
+    (total bytes >= 4x the L2 size) is swept by a CUDA graph of back-to-back
+    launches, so every launch streams its weight from HBM.
+    Returns {shape: {M: {us, GBs, frac}}} with algorithmic bytes per call:
+    W^_q + its E8M0 + Q(R) + its E8M0 + token codes and scales + bf16 Y.
+    """
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import workload
+    wl = workload("decode_mxfp4")
+    l2 = torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+    hbm = measured_peaks()[0]["hbm_gbs"]
+    out = {}
+    for lin in wl.linears:
+        K, N, r = lin.K, lin.N, lin.r
+        rp = ((r + 63) // 64) * 64 if r else 0
+        W = torch.from_numpy(lin.W()).to(torch.bfloat16).cuda()
+        a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(16)).to(torch.bfloat16).cuda())
+        w_bytes = N * K // 2 + N * K // 32 + N * rp // 2 + N * rp // 32
+        n_pool = max(2, -(-4 * l2 // w_bytes))
+        pool = [S.serq_prepare(W, r, lin.fmt, act_absmax=a) for _ in range(n_pool)]
+        del W
+        out[lin.name] = {"K": K, "N": N, "pool": n_pool}
+        for M in tokens:
+            X = torch.from_numpy(lin.X(M)).to(torch.bfloat16).cuda()
+            qa = S.serq_quant_act(S.serq_fold_producer(pool[0], X), r, lin.fmt)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            for w in pool:
+                S.serq_linear(w, qa, Y=Y)
+            torch.cuda.synchronize()
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                for w in pool:
+                    S.serq_linear(w, qa, Y=Y)
+            g.replay()
+            g.replay()
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record()
+            for _ in range(reps):
+                g.replay()
+            end.record()
+            torch.cuda.synchronize()
+            S.serq_device_status()
+            t = start.elapsed_time(end) * 1e-3 / (reps * n_pool)
+            nbytes = w_bytes + M * (K // 2 + K // 32 + rp // 2 + rp // 32) + 2 * M * N
+            out[lin.name][f"M{M}"] = {"us": round(t * 1e6, 3), "GBs": round(nbytes / t / 1e9, 1),
+                                      "frac": round(nbytes / t / 1e9 / hbm, 3)}
+            del g
+        del pool
+        torch.cuda.empty_cache()
+    return out
+
+
 # ----------------------------------------------------------------- CPU oracle
 def cpu_oracle_prepare(wl, r_override=None):
     """The oracle's offline preparation of every linear (not timed)."""
@@ -416,6 +472,11 @@ def main():
                               "serq_linear_us": g2[0] * 1e3,
                               "frac_of_int8_peak": f2 / (g2[0] * 1e-3) / 1e12 / (peaks["bf16_tflops_sustained"] * 2)}
         del layers2
+    if not args.no_extras and rank == 0:
+        dec = bench_decode()
+        line["decode"] = dec
+        m16 = [v["M16"]["GBs"] for v in dec.values() if isinstance(v, dict) and "M16" in v]
+        line["decode_GBs_M16_mean"] = sum(m16) / len(m16)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, flops, cores = cpu_oracle_step(cpu_oracle_prepare(wl), args.cpu_rows)
         line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",

@@ -90,3 +90,34 @@ def test_residual_reduces_error_on_gpu():
     ref = X.astype(np.float64) @ W.astype(np.float64)
     errs = [np.linalg.norm(run_gpu(X, W, r, "int4")["Y"] - ref) for r in (0, 16, 64)]
     assert errs[1] < errs[0] and errs[2] < errs[1]
+
+
+@pytest.mark.parametrize("M,K,N,r", [
+    (1, 4096, 1024, 128),     # the pages' rank, k/v shape at one token
+    (4, 1024, 512, 128),      # 5 K-tiles over 5 splits
+    (8, 512, 256, 64),
+    (9, 768, 384, 0),         # r = 0, 16-token MMA with 7 padding tokens
+    (16, 4096, 1024, 256),
+    (16, 256, 128, 256),      # one K-tile each for main and residual
+])
+def test_decode_shapes(M, K, N, r):
+    # small M takes the split-K streaming kernel (MXFP4)
+    X = activations(3000 + M, M, K, max(1, K // 100), "const", 50.0)
+    Xc = activations(3100 + M, 256, K, max(1, K // 100), "const", 50.0)
+    W = weights(3200 + K, K, N)
+    _check(X, W, r, "mxfp4", X_calib=Xc)
+
+
+def test_decode_repeated_calls_identical():
+    # the split-K tickets are reset by each call: repeated calls agree bit for bit
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from parity_util import to_dev_bf16
+    M, K, N, r = 16, 2048, 512, 128
+    X = activations(41, M, K, 20, "const", 50.0)
+    W = weights(42, K, N)
+    w = S.serq_prepare(to_dev_bf16(W), r, "mxfp4", act_absmax=S.serq_calib_absmax(to_dev_bf16(X)))
+    qa = S.serq_quant_act(S.serq_fold_producer(w, to_dev_bf16(X)), r, "mxfp4")
+    ys = [S.serq_linear(w, qa).clone() for _ in range(3)]
+    S.serq_device_status()
+    assert all(torch.equal(ys[0], y) for y in ys[1:])

@@ -1,0 +1,233 @@
+// serq_linear, MXFP4, small M (decode; M <= 16): the same product as the
+// prefill kernel, organised to stream W^_q and Q(R) from HBM at full rate.
+//
+//  * swap-AB: the weight tile (128 output channels) is the MMA's A operand
+//    (M_mma = 128) and the <= 16 tokens are its B operand (N_mma = 8 or 16),
+//    so no tensor-core rows are spent on padding tokens;
+//  * split-K: the K-tiles of the main product followed by the residual's
+//    K-tiles ("量化推理": one extra r x N product, no intermediate
+//    quantization) are cut into S contiguous ranges; CTA (n_blk, split)
+//    streams 128 weight rows over its range;
+//  * each CTA writes fp32 partial sums to a workspace; the last CTA of an
+//    output block (ticket counter) adds the S partials in split order (a
+//    fixed order, so results do not depend on scheduling), writes bf16 Y and
+//    resets the counter for the next call.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "gemm_mxfp4.cuh"
+
+namespace serq {
+namespace mxd {
+
+constexpr int BM = 128;                 // output channels per CTA
+constexpr int BK = 256;                 // codes per K-tile
+constexpr int BK_BYTES = 128;
+constexpr int MAX_TOKENS = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB weight codes
+constexpr int B_BYTES = MAX_TOKENS * BK_BYTES;   // 2 KB token codes
+constexpr int SFA_BYTES = 2 * 512;               // weight scale atoms
+constexpr int SFB_BYTES = 2 * 512;               // token scale atoms
+constexpr int THREADS = 64 + 4 * 32;             // producer, MMA, 4 epilogue warps
+constexpr uint32_t TMEM_COLS = 32;
+constexpr uint32_t TMEM_ACC = 0;                 // 16 fp32 columns (tokens)
+constexpr uint32_t TMEM_SFA = 16;                // 2 atoms x 4 columns
+constexpr uint32_t TMEM_SFB = 24;                // 2 atoms x 4 columns
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 1024 + 256;
+
+}  // namespace mxd
+
+struct MxDecodeParams {
+    int M, N, K, rp;
+    int n_tokens_mma;       // 8 or 16
+    int k_tiles_main, k_tiles_total;
+    int splits;
+    int atoms_k_main, atoms_k_res;
+    const uint8_t* sf_w;    // weight scale atoms (main)
+    const uint8_t* sf_x;    // token scale atoms (main)
+    const uint8_t* sf_wr;   // residual scale atoms
+    const uint8_t* sf_xr;   // salient-slice scale atoms
+    float* partial;         // [splits][M][N] workspace
+    unsigned int* tickets;  // [N / 128], zero between calls
+    __nv_bfloat16* Y;
+};
+
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),
+          "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+__global__ void __launch_bounds__(mxd::THREADS)
+serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
+                                const __grid_constant__ CUtensorMap tm_wr, const __grid_constant__ CUtensorMap tm_xr,
+                                const MxDecodeParams p) {
+    using namespace mxd;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * A_BYTES;
+    uint8_t* sSFA = sB + STAGES * B_BYTES;
+    uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+    uint64_t* empty = full + STAGES;
+    uint64_t* acc_full = empty + STAGES;
+    uint64_t* drain = acc_full + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    __shared__ unsigned int s_is_last;
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const int n_blk = blockIdx.x;
+    const int split = blockIdx.y;
+    const int kt0 = static_cast<int>((static_cast<long long>(p.k_tiles_total) * split) / p.splits);
+    const int kt1 = static_cast<int>((static_cast<long long>(p.k_tiles_total) * (split + 1)) / p.splits);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], 1);
+        }
+        mbar_init(acc_full, 1);
+        mbar_init(drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            for (int kt = kt0; kt < kt1; ++kt) {
+                if (!mbar_wait(&empty[s], ph ^ 1u, 0x121u)) break;
+                const bool res = kt >= p.k_tiles_main;
+                const int kk = res ? kt - p.k_tiles_main : kt;
+                const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
+                const int na = min(2, atoms - 2 * kk);
+                mbar_arrive_expect_tx(&full[s], A_BYTES + p.n_tokens_mma * BK_BYTES + 2u * na * 512u);  // token box = n_tokens_mma rows
+                tma_load_2d(sA + s * A_BYTES, res ? &tm_wr : &tm_w, &full[s], kk * BK_BYTES, n_blk * BM);
+                tma_load_2d(sB + s * B_BYTES, res ? &tm_xr : &tm_x, &full[s], kk * BK_BYTES, 0);
+                bulk_load(sSFA + s * SFA_BYTES,
+                          (res ? p.sf_wr : p.sf_w) + (static_cast<size_t>(n_blk) * atoms + 2 * kk) * 512, na * 512,
+                          &full[s]);
+                bulk_load(sSFB + s * SFB_BYTES, (res ? p.sf_xr : p.sf_x) + static_cast<size_t>(2 * kk) * 512,
+                          na * 512, &full[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            // every stage released (all tensor-core reads and barrier arrivals done)
+            for (int i = 0; i < STAGES; ++i) {
+                if (!mbar_wait(&empty[s], ph ^ 1u, 0x122u)) break;
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            const uint32_t id_even = idesc_mxf4(BM, p.n_tokens_mma, 0, 0);
+            const uint32_t id_odd = idesc_mxf4(BM, p.n_tokens_mma, 2, 2);
+            bool first = true;
+            for (int kt = kt0; kt < kt1; ++kt) {
+                if (!mbar_wait(&full[s], ph, 0x221u)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const bool res = kt >= p.k_tiles_main;
+                const int kk = res ? kt - p.k_tiles_main : kt;
+                const int width = res ? p.rp : p.K;
+                const int steps = min(4, (width - kk * BK) / 64);
+                const int na = (steps + 1) / 2;
+                const uint32_t a_base = smem_u32(sA + s * A_BYTES);
+                const uint32_t b_base = smem_u32(sB + s * B_BYTES);
+                const uint32_t sfa_base = smem_u32(sSFA + s * SFA_BYTES);
+                const uint32_t sfb_base = smem_u32(sSFB + s * SFB_BYTES);
+                for (int j = 0; j < na; ++j) {
+                    tc_cp_32x128b_warpx4(tmem + TMEM_SFA + 4 * j, sdesc_sf_atom(sfa_base + 512 * j));
+                    tc_cp_32x128b_warpx4(tmem + TMEM_SFB + 4 * j, sdesc_sf_atom(sfb_base + 512 * j));
+                }
+                for (int st = 0; st < steps; ++st) {
+                    tc_mma_mxf4(tmem + TMEM_ACC, sdesc_kmajor_sw128(a_base + 32 * st),
+                                sdesc_kmajor_sw128(b_base + 32 * st), (st & 1) ? id_odd : id_even,
+                                tmem + TMEM_SFA + 4 * (st >> 1), tmem + TMEM_SFB + 4 * (st >> 1), first ? 0u : 1u);
+                    first = false;
+                }
+                tc_commit(&empty[s]);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+            if (ok) tc_commit(acc_full);
+            tc_commit(drain);
+            mbar_wait(drain, 0, 0x222u);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue: partial sums
+        const int quad = warp & 3;
+        const int n = n_blk * BM + quad * 32 + lane;
+        if (__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, 0x321u))) {
+            tc_fence_after();
+            uint32_t v[16];
+            tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TMEM_ACC, v);
+            tmem_ld_wait();
+            float* part = p.partial + static_cast<size_t>(split) * p.M * p.N;
+#pragma unroll
+            for (int m = 0; m < MAX_TOKENS; ++m)
+                if (m < p.M) part[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[m]);
+        }
+        tc_fence_before();
+    }
+
+    // ---------------------------------------------------------------- split reduction
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const unsigned int ticket = atomicAdd(&p.tickets[n_blk], 1u);
+        s_is_last = (ticket == static_cast<unsigned int>(p.splits - 1)) ? 1u : 0u;
+    }
+    __syncthreads();
+    if (s_is_last) {
+        __threadfence();
+        for (int idx = threadIdx.x; idx < p.M * BM; idx += blockDim.x) {
+            const int m = idx / BM;
+            const int n = n_blk * BM + idx % BM;
+            float acc = 0.0f;
+            for (int sp = 0; sp < p.splits; ++sp)
+                acc += __ldcg(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n);
+            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc);
+        }
+        if (threadIdx.x == 0) p.tickets[n_blk] = 0u;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace serq

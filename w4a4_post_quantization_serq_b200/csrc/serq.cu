@@ -19,6 +19,7 @@
 #include "prepare.cuh"
 #include "gemm_mxfp4.cuh"
 #include "gemm_int4.cuh"
+#include "gemm_mxfp4_decode.cuh"
 
 using namespace serq;
 
@@ -65,7 +66,20 @@ struct DeviceInfo {
     int sms = 0;
     bool smem_set_mx = false;
     bool smem_set_i4 = false;
+    bool smem_set_mxd = false;
 };
+
+// split-K ranges of the small-M kernel: about two CTAs per SM, at most
+// kMaxDecodeSplits, never more than the number of K-tiles
+constexpr int kMaxDecodeSplits = 8;
+constexpr int kMaxDecodeTokens = 16;
+
+int decode_splits(int n_blocks, int k_tiles, int sms) {
+    int s = (2 * sms + n_blocks - 1) / n_blocks;
+    if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
+    if (s > k_tiles) s = k_tiles;
+    return s < 1 ? 1 : s;
+}
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
 
@@ -145,8 +159,12 @@ struct serq_weight {
     size_t rq_bytes;
     void* rsc;
     size_t rsc_bytes;
-    CUtensorMap tm_w;
+    CUtensorMap tm_w;      // B operand of the prefill kernels (256-row boxes)
     CUtensorMap tm_r;
+    CUtensorMap tm_w128;   // A operand of the small-M kernel (128-row boxes, MXFP4)
+    CUtensorMap tm_r128;
+    float* dec_partial;    // small-M split-K workspace [kMaxDecodeSplits][16][N] (MXFP4)
+    unsigned int* dec_tickets;  // [N / 128], zero between calls
 };
 
 extern "C" {
@@ -246,6 +264,9 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     const size_t o_perm = take(4u * K), o_s = take(4u * K), o_sp = take(4u * K), o_inv = take(4u * K);
     const size_t o_wq = take(w->wq_bytes), o_wsc = take(w->wsc_bytes);
     const size_t o_rq = take(w->rq_bytes), o_rsc = take(w->rsc_bytes);
+    const bool mx = fmt == SERQ_FMT_MXFP4;
+    const size_t o_dp = take(mx ? sizeof(float) * kMaxDecodeSplits * kMaxDecodeTokens * static_cast<size_t>(N) : 0);
+    const size_t o_dt = take(mx ? 4u * (N / 128) : 0);
     const size_t keep = off;
     const size_t o_b = take(4u * K), o_col = take(4u * N);
     void* arena = nullptr;
@@ -266,6 +287,8 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     w->wsc = base + o_wsc;
     w->rq = base + o_rq;
     w->rsc = base + o_rsc;
+    w->dec_partial = mx ? reinterpret_cast<float*>(base + o_dp) : nullptr;
+    w->dec_tickets = mx ? reinterpret_cast<unsigned int*>(base + o_dt) : nullptr;
     float* tmp_b = reinterpret_cast<float*>(base + o_b);
     unsigned int* tmp_col = reinterpret_cast<unsigned int*>(base + o_col);
 
@@ -322,6 +345,14 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
         if (serq_status st = make_map(&w->tm_r, w->rq, rp / 2, N, bi, 256, swz)) return bail(st);
     } else {
         w->tm_r = w->tm_w;
+    }
+    if (mx) {
+        if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return bail(st);
+        if (rp > 0) {
+            if (serq_status st = make_map(&w->tm_r128, w->rq, rp / 2, N, 128, 128, true)) return bail(st);
+        } else {
+            w->tm_r128 = w->tm_w128;
+        }
     }
 #undef PREP_CUDA
     *out = w;
@@ -420,6 +451,46 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
     const int K = w->K, N = w->N, rp = w->rp;
+    if (w->fmt == SERQ_FMT_MXFP4 && M <= kMaxDecodeTokens) {
+        const int n_tok = M <= 8 ? 8 : 16;
+        CUtensorMap tm_x, tm_xr;
+        if (serq_status st = make_map(&tm_x, xq, K / 2, M, 128, n_tok, true)) return st;
+        if (rp > 0) {
+            if (serq_status st = make_map(&tm_xr, xsq, rp / 2, M, 128, n_tok, true)) return st;
+        } else {
+            tm_xr = tm_x;
+        }
+        if (!info->smem_set_mxd) {
+            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, mxd::SMEM_BYTES));
+            info->smem_set_mxd = true;
+        }
+        MxDecodeParams p;
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.rp = rp;
+        p.n_tokens_mma = n_tok;
+        p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
+        p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
+        const int n_blocks = N / mxd::BM;
+        p.splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
+        p.atoms_k_main = K / 128;
+        p.atoms_k_res = (rp + 127) / 128;
+        p.sf_w = static_cast<const uint8_t*>(w->wsc);
+        p.sf_x = static_cast<const uint8_t*>(xs);
+        p.sf_wr = static_cast<const uint8_t*>(w->rsc);
+        p.sf_xr = static_cast<const uint8_t*>(xss);
+        p.partial = w->dec_partial;
+        p.tickets = w->dec_tickets;
+        p.Y = static_cast<__nv_bfloat16*>(Y);
+        const dim3 grid(n_blocks, p.splits);
+        serq_linear_mxfp4_decode_kernel<<<grid, mxd::THREADS, mxd::SMEM_BYTES, cs>>>(w->tm_w128, tm_x, w->tm_r128,
+                                                                                      tm_xr, p);
+        SERQ_CUDA(cudaGetLastError());
+        return SERQ_OK;
+    }
+
     const uint32_t bi = box_inner_bytes(w->fmt);
     const bool swz = w->fmt == SERQ_FMT_MXFP4;
     CUtensorMap tm_a, tm_ar;
