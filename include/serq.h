@@ -178,6 +178,43 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
                         const void* xsq, const void* xss, void* Y, int32_t* acc_dbg,
                         serq_stream stream);
 
+/* ------------------------------------------------------------------------
+ * serq_linear_small_m_noalloc — the small-M (M <= 16) MXFP4 linear for
+ * callers that cannot allocate device memory. (The SERQ paper has no
+ * counterpart; this is an interface addition of this library.)
+ *
+ * Who needs it: runtimes that plan every device buffer ahead of time and do
+ * not allow cudaMalloc on the serving path (cudaMalloc can synchronize the
+ * device and can fail under memory pressure), and code that holds packed
+ * weights in memory it manages itself rather than in a serq_weight. Such a
+ * caller passes every input and the output as raw device pointers; the call
+ * allocates nothing (no cudaMalloc/cudaFree, no allocating library routine).
+ *
+ * Inputs, in the layouts of include/serq.h (for example the buffers that
+ * serq_weight_get_view returns for an MXFP4 weight, and serq_quant_act's
+ * outputs for the same M, K, r): wq u8[N][K/2], w_scale E8M0 atoms
+ * (N rows, K/32 blocks), rq u8[N][rp/2], r_scale E8M0 atoms (N rows, rp/32
+ * blocks), xq/xs/xsq/xss. rq, r_scale, xsq and xss may be NULL when r == 0.
+ * Output: Y bf16 [M][N]. Same result as serq_linear for the same operands.
+ *
+ * Scratch: the split-K partial sums and tickets of the small-M kernel live
+ * in one static device array of 4 MiB inside the library (held by every GPU
+ * that loads the library until the process exits). Limits: 1 <= M <= 16,
+ * N <= 131072 (the ticket area) and M*N <= 1047552 (the partial-sum area);
+ * larger sizes return SERQ_EINVAL with the limit in serq_last_error(). The
+ * number of K splits shrinks when M*N leaves room for fewer.
+ * Every call shares the array and it keeps the last call's contents (each
+ * call clears the tickets it uses, on `stream`, before its kernel): calls
+ * that overlap on the GPU (other streams, other host threads) race.
+ * The first call on a device does a one-time set-up (it looks up the
+ * array's device address with cudaGetSymbolAddress); make that first call
+ * before any stream capture. Asynchronous on `stream`.
+ * Errors: EINVAL, EUNSUPPORTED, ECUDA.
+ * ------------------------------------------------------------------------ */
+serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* wq, const void* w_scale,
+                                        const void* rq, const void* r_scale, const void* xq, const void* xs,
+                                        const void* xsq, const void* xss, void* Y, serq_stream stream);
+
 /* Synchronizes the stream, then reports (and clears) any device-side pipeline
  * timeout recorded by this library's kernels on the current device:
  * SERQ_ETIMEOUT if one occurred since the last call, else SERQ_OK

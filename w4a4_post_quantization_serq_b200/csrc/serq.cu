@@ -167,6 +167,33 @@ struct serq_weight {
     unsigned int* dec_tickets;  // [N / 128], zero between calls
 };
 
+// ============================================================== allocation-free small-M entry
+// Scratch of serq_linear_small_m_noalloc: split-K tickets (first 4 KiB, one
+// uint32 per 128 output channels) followed by fp32 partial sums. It lives in
+// the library image, so every GPU that loads the library holds it until exit.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+constexpr size_t kNoAllocTicketBytes = 4096;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mu;
+
+// Device address of the scratch array on the current device, looked up once
+// per device (host code only holds a stand-in symbol, not a device address).
+serq_status noalloc_scratch(int dev, void** out) {
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(g_noalloc_scratch)");
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return SERQ_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char* serq_last_error(void) { return g_last_error.c_str(); }
@@ -551,6 +578,79 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.acc_dbg = acc_dbg;
         serq_linear_int4_kernel<<<grid, i4::THREADS, i4::SMEM_BYTES, cs>>>(tm_a, w->tm_w, tm_ar, w->tm_r, p);
     }
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
+serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* wq, const void* w_scale,
+                                        const void* rq, const void* r_scale, const void* xq, const void* xs,
+                                        const void* xsq, const void* xss, void* Y, serq_stream stream) {
+    if (M < 1 || M > kMaxDecodeTokens) return fail(SERQ_EINVAL, "M=%d outside 1..%d", M, kMaxDecodeTokens);
+    if (K < 128 || K % 128 != 0 || K > 32768 || N < 128 || N % 128 != 0 || r < 0 || r > K)
+        return fail(SERQ_EINVAL, "bad shape K=%d N=%d r=%d (need K%%128==0, K<=32768, N%%128==0, 0<=r<=K)", K, N, r);
+    if (static_cast<size_t>(N / 128) * 4u > kNoAllocTicketBytes)
+        return fail(SERQ_EINVAL, "N=%d above the static scratch limit of %zu output channels", N,
+                    kNoAllocTicketBytes / 4u * 128u);
+    const size_t cap_floats = (kNoAllocScratchBytes - kNoAllocTicketBytes) / sizeof(float);
+    if (static_cast<size_t>(M) * N > cap_floats)
+        return fail(SERQ_EINVAL, "M*N=%zu above the static scratch limit of %zu", static_cast<size_t>(M) * N,
+                    cap_floats);
+    const int rp = residual_width(r);
+    if (wq == nullptr || w_scale == nullptr || xq == nullptr || xs == nullptr || Y == nullptr)
+        return fail(SERQ_EINVAL, "NULL pointer");
+    if (rp > 0 && (rq == nullptr || r_scale == nullptr || xsq == nullptr || xss == nullptr))
+        return fail(SERQ_EINVAL, "r > 0 needs rq, r_scale, xsq and xss");
+    if (!aligned16(wq) || !aligned16(w_scale) || !aligned16(xq) || !aligned16(xs) || !aligned16(Y) ||
+        (rp > 0 && (!aligned16(rq) || !aligned16(r_scale) || !aligned16(xsq) || !aligned16(xss))))
+        return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    void* scratch = nullptr;
+    if (serq_status st = noalloc_scratch(dev, &scratch)) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+    const int n_tok = M <= 8 ? 8 : 16;
+    CUtensorMap tm_w, tm_wr, tm_x, tm_xr;
+    if (serq_status st = make_map(&tm_w, wq, K / 2, N, 128, 128, true)) return st;
+    if (serq_status st = make_map(&tm_x, xq, K / 2, M, 128, n_tok, true)) return st;
+    if (rp > 0) {
+        if (serq_status st = make_map(&tm_wr, rq, rp / 2, N, 128, 128, true)) return st;
+        if (serq_status st = make_map(&tm_xr, xsq, rp / 2, M, 128, n_tok, true)) return st;
+    } else {
+        tm_wr = tm_w;
+        tm_xr = tm_x;
+    }
+    if (!info->smem_set_mxd) {
+        SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       mxd::SMEM_BYTES));
+        info->smem_set_mxd = true;
+    }
+    MxDecodeParams p;
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.rp = rp;
+    p.n_tokens_mma = n_tok;
+    p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
+    p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
+    const int n_blocks = N / mxd::BM;
+    int splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
+    while (splits > 1 && static_cast<size_t>(splits) * M * N > cap_floats) --splits;
+    p.splits = splits;
+    p.atoms_k_main = K / 128;
+    p.atoms_k_res = (rp + 127) / 128;
+    p.sf_w = static_cast<const uint8_t*>(w_scale);
+    p.sf_x = static_cast<const uint8_t*>(xs);
+    p.sf_wr = static_cast<const uint8_t*>(r_scale);
+    p.sf_xr = static_cast<const uint8_t*>(xss);
+    p.tickets = static_cast<unsigned int*>(scratch);
+    p.partial = reinterpret_cast<float*>(static_cast<unsigned char*>(scratch) + kNoAllocTicketBytes);
+    p.Y = static_cast<__nv_bfloat16*>(Y);
+    // the array keeps the previous call's contents: the tickets must start at zero
+    SERQ_CUDA(cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(n_blocks) * sizeof(unsigned int), cs));
+    serq_linear_mxfp4_decode_kernel<<<dim3(n_blocks, splits), mxd::THREADS, mxd::SMEM_BYTES, cs>>>(tm_w, tm_x, tm_wr,
+                                                                                                  tm_xr, p);
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
 }

@@ -164,6 +164,21 @@ def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
     return Y
 
 
+def serq_linear_small_m_noalloc(M: int, K: int, N_: int, r: int, wq: torch.Tensor, w_scale: torch.Tensor,
+                                rq: Optional[torch.Tensor], r_scale: Optional[torch.Tensor], qa: QuantAct,
+                                Y: torch.Tensor, stream=None) -> torch.Tensor:
+    """Small-M MXFP4 linear from caller-owned buffers only; the library allocates nothing.
+
+    For callers that cannot allocate device memory on their serving path: the
+    split-K scratch lives in a static device array of the library (calls that
+    overlap on the GPU race on it). Output Y must be preallocated (bf16 M x N).
+    """
+    N.check(N.load().serq_linear_small_m_noalloc(M, K, N_, r, _ptr(wq), _ptr(w_scale), _ptr(rq), _ptr(r_scale),
+                                                 _ptr(qa.xq), _ptr(qa.xs), _ptr(qa.xsq), _ptr(qa.xss), _ptr(Y),
+                                                 _stream(stream)))
+    return Y
+
+
 def serq_device_status(stream=None) -> None:
     """Synchronize and raise SerqError(SERQ_ETIMEOUT) if a kernel wait timed out."""
     N.check(N.load().serq_device_status(_stream(stream)))
