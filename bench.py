@@ -31,6 +31,7 @@ METRIC = "serq_linear TOPS (2·M·N·(K+r)/t) and % of FP4 peak; decode GB/s; ov
 WORKLOAD = "mlp_mxfp4"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
 CAPTURED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+DOMINANT_KERNEL = "serq_linear_mxfp4_pair_kernel"  # M > 128 MXFP4 prefill (CTA pairs)
 
 
 def parse_args():
@@ -352,11 +353,13 @@ def captured_traffic():
     import hashlib
     try:
         rec = json.load(open(CAPTURED_TRAFFIC_FILE))
-        src = os.path.join(ROOT, "w4a4_post_quantization_serq_b200", "csrc", "gemm_mxfp4.cuh")
+        src = os.path.join(ROOT, "w4a4_post_quantization_serq_b200", "csrc", rec.get("source", "gemm_mxfp4.cuh"))
         sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
     except (OSError, ValueError):
         return None
-    return rec.get("dram_bytes_per_launch") if rec.get("source_sha256_prefix") == sha else None
+    if rec.get("source_sha256_prefix") != sha or rec.get("kernel") != DOMINANT_KERNEL:
+        return None
+    return rec.get("dram_bytes_per_launch")
 
 
 def reference_main(args, world, rank, pg):
@@ -428,7 +431,7 @@ def main():
     traffic = captured_traffic()
     roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak, "traffic": traffic,
-                "kernel": "serq_linear_mxfp4_kernel", "launch": layers[dom]["lin"].name,
+                "kernel": DOMINANT_KERNEL, "launch": layers[dom]["lin"].name,
                 "flops_per_launch": layers[dom]["flops"],
                 "peak_source": f"{peak_src} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
                                f"{FP4_OVER_BF16:g} (nominal dense FP4/BF16 ratio)",

@@ -51,6 +51,9 @@ def test_tiny_workload(fmt):
     (64, 512, 256, 256),      # r = 256
     (129, 768, 1280, 40),     # r not a multiple of 32 (short salient block)
     (33, 256, 256, 256),      # r = K
+    (300, 512, 512, 64),      # MXFP4 CTA pair whose second CTA has no rows (M % 256 <= 128)
+    (257, 384, 384, 32),      # CTA pair with a half K-tile and a half N-tile
+    (1024, 1024, 1536, 128),  # several pair tiles per cluster
 ])
 def test_shapes(fmt, M, K, N, r):
     X = activations(1000 + M, M, K, max(1, K // 100), "lognormal", 50.0)

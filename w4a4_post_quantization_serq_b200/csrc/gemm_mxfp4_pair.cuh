@@ -1,0 +1,317 @@
+// serq_linear, MXFP4, prefill on a CTA pair (cluster of 2, tcgen05 cta_group::2).
+//
+// Same product as serq_linear_mxfp4_kernel ("量化推理": main K-tiles, then the
+// residual's K-tiles, one fp32 accumulator), on a 256 x 256 output tile per
+// CTA pair. Each CTA loads its own 128 rows of A and its own 128-row half of
+// B; one thread of the even CTA issues M = 256 MMAs that read both CTAs'
+// shared memory and write each CTA's 128 rows of D into that CTA's tensor
+// memory. Per CTA, a K-tile stage is 35 KB instead of the 51 KB of the
+// single-CTA 128 x 256 tile, so the shared-memory traffic of the tensor core
+// plus TMA fits the shared-memory port, and six stages fit.
+//
+// Warp roles (each CTA): 0 TMA producer; 1 TMEM owner (+ MMA issuer in the
+// even CTA); 2 bridge (waits this CTA's stage, arrives on the even CTA's
+// "ready" barrier); 3..10 epilogue (tcgen05.ld -> release -> bf16 -> store).
+//
+// Two accumulators alternate between tiles so the epilogue of one tile
+// overlaps the MMAs of the next. Two 256-column fp32 tiles and the scale
+// factors do not fit the 512 tensor-memory columns, so the buffers overlap in
+// 24 columns: [0, 256) and [232, 488), scales in [488, 512). The epilogue
+// drains the shared columns [232, 256) first and signals "overlap free"; the
+// next tile's MMAs wait only for that signal (and for their own buffer's
+// previous tile to be fully drained).
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "gemm_mxfp4.cuh"
+
+namespace serq {
+namespace mxp {
+
+constexpr int BM = 128;                       // rows of A per CTA (pair tile: 256)
+constexpr int BN = 256;                       // output channels per pair tile
+constexpr int BN_HALF = 128;                  // rows of B per CTA
+constexpr int BK_BYTES = 128;
+constexpr int BK = 256;
+constexpr int STAGES = 6;
+constexpr int A_BYTES = BM * BK_BYTES;        // 16 KB
+constexpr int B_BYTES = BN_HALF * BK_BYTES;   // 16 KB
+constexpr int SFA_BYTES = 2 * 512;            // own 128 rows x 8 scales
+constexpr int SFB_BYTES = 4 * 512;            // all 256 rows x 8 scales
+constexpr int NUM_EPI_WARPS = 8;
+constexpr int EPI_WARP0 = 3;
+constexpr int THREADS = (EPI_WARP0 + NUM_EPI_WARPS) * 32;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_ACC0 = 0;
+constexpr uint32_t TMEM_ACC1 = 232;           // shares columns [232, 256) with buffer 0
+constexpr uint32_t OVL_LO = 232;              // first shared column
+constexpr uint32_t TMEM_SFA = 488;
+constexpr uint32_t TMEM_SFB = 496;
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 1024 + 256;
+
+}  // namespace mxp
+
+struct MxPairParams {
+    int M, N, K, rp;
+    int num_n_tiles, num_tiles;     // pair tiles, n fastest
+    int k_tiles_main, k_tiles_res;
+    int atoms_k_main, atoms_k_res;
+    int row_blocks_a;               // ceil(M / 128): activation scale atoms that exist
+    const uint8_t* sfa;
+    const uint8_t* sfb;
+    const uint8_t* sfa_r;
+    const uint8_t* sfb_r;
+    __nv_bfloat16* Y;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mxp::THREADS, 1)
+serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
+                              const __grid_constant__ CUtensorMap tm_ar, const __grid_constant__ CUtensorMap tm_br,
+                              const MxPairParams p) {
+    using namespace mxp;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = sA + STAGES * A_BYTES;
+    uint8_t* sSFA = sB + STAGES * B_BYTES;
+    uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);  // this CTA's loads landed
+    uint64_t* ready = full + STAGES;      // even CTA: both CTAs' loads landed
+    uint64_t* empty = ready + STAGES;     // stage consumed (multicast commit)
+    uint64_t* acc_full = empty + STAGES;  // [2] accumulator complete (multicast commit)
+    uint64_t* acc_empty = acc_full + 2;   // [2] even CTA: both epilogues drained the accumulator
+    uint64_t* ovl_empty = acc_empty + 2;  // even CTA: both epilogues drained the shared columns
+    uint64_t* drain = ovl_empty + 1;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+    const uint32_t rank = cluster_ctarank();
+    const bool leader = rank == 0;
+    const int cluster = blockIdx.x >> 1;
+    const int num_clusters = gridDim.x >> 1;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&ready[s], 2);
+            mbar_init(&empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 2 * NUM_EPI_WARPS * 32);
+        }
+        mbar_init(ovl_empty, 2 * 4 * 32);  // the four warps that own the shared columns, both CTAs
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_a);
+        tma_prefetch_desc(&tm_b);
+        if (p.k_tiles_res > 0) {
+            tma_prefetch_desc(&tm_ar);
+            tma_prefetch_desc(&tm_br);
+        }
+    }
+    cluster_sync();
+    if (warp == 1) {
+        tmem_alloc_pair(tmem_slot, TMEM_COLS);
+        tmem_relinquish_pair();
+    }
+    tc_fence_before();
+    cluster_sync();  // barriers of both CTAs initialised, TMEM of both allocated
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const int total_k = p.k_tiles_main + p.k_tiles_res;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = cluster; tile < p.num_tiles && ok; tile += num_clusters) {
+                const int n_blk = tile % p.num_n_tiles;
+                const int m_pair = tile / p.num_n_tiles;
+                const int a_rowblk = 2 * m_pair + static_cast<int>(rank);
+                const bool a_sf = a_rowblk < p.row_blocks_a;
+                const bool hi_half = (n_blk * BN + 128) < p.N;
+                for (int kt = 0; kt < total_k; ++kt) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, 0x131u)) {
+                        ok = false;
+                        break;
+                    }
+                    const bool res = kt >= p.k_tiles_main;
+                    const int kk = res ? kt - p.k_tiles_main : kt;
+                    const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
+                    const int na = min(2, atoms - 2 * kk);
+                    const uint8_t* sfa_src = res ? p.sfa_r : p.sfa;
+                    const uint8_t* sfb_src = res ? p.sfb_r : p.sfb;
+                    const uint32_t sf_bytes = static_cast<uint32_t>(na * 512) * ((a_sf ? 1u : 0u) + (hi_half ? 2u : 1u));
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes);
+                    tma_load_2d(sA + s * A_BYTES, res ? &tm_ar : &tm_a, &full[s], kk * BK_BYTES, a_rowblk * BM);
+                    tma_load_2d(sB + s * B_BYTES, res ? &tm_br : &tm_b, &full[s], kk * BK_BYTES,
+                                n_blk * BN + static_cast<int>(rank) * BN_HALF);
+                    if (a_sf)
+                        bulk_load(sSFA + s * SFA_BYTES,
+                                  sfa_src + (static_cast<size_t>(a_rowblk) * atoms + 2 * kk) * 512, na * 512, &full[s]);
+                    bulk_load(sSFB + s * SFB_BYTES,
+                              sfb_src + (static_cast<size_t>(2 * n_blk) * atoms + 2 * kk) * 512, na * 512, &full[s]);
+                    if (hi_half)
+                        bulk_load(sSFB + s * SFB_BYTES + 1024,
+                                  sfb_src + (static_cast<size_t>(2 * n_blk + 1) * atoms + 2 * kk) * 512, na * 512,
+                                  &full[s]);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            for (int i = 0; i < STAGES && ok; ++i) {
+                ok = mbar_wait(&empty[s], ph ^ 1u, 0x132u);
+                if (++s == STAGES) {
+                    s = 0;
+                    ph ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 2) {
+        // ------------------------------------------------------------ bridge (both CTAs)
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            for (int tile = cluster; tile < p.num_tiles && ok; tile += num_clusters) {
+                for (int kt = 0; kt < total_k; ++kt) {
+                    if (!mbar_wait(&full[s], ph, 0x133u)) {
+                        ok = false;
+                        break;
+                    }
+                    mbar_arrive_cluster(&ready[s], 0);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer (even CTA)
+        if (leader && lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            bool ok = true;
+            const uint32_t id_even = idesc_mxf4(2 * BM, BN, 0, 0);
+            const uint32_t id_odd = idesc_mxf4(2 * BM, BN, 2, 2);
+            int it = 0;  // tiles issued by this pair so far
+            for (int tile = cluster; tile < p.num_tiles && ok; tile += num_clusters, ++it) {
+                const int b = it & 1;
+                // this buffer's previous tile fully drained, and the shared columns of the previous tile
+                if (!mbar_wait_cluster(&acc_empty[b], static_cast<uint32_t>(((it >> 1) & 1) ^ 1), 0x231u) ||
+                    (it > 0 && !mbar_wait_cluster(ovl_empty, static_cast<uint32_t>((it - 1) & 1), 0x234u))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t acc_col = b ? TMEM_ACC1 : TMEM_ACC0;
+                for (int kt = 0; kt < total_k; ++kt) {
+                    if (!mbar_wait_cluster(&ready[s], ph, 0x232u)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const bool res = kt >= p.k_tiles_main;
+                    const int kk = res ? kt - p.k_tiles_main : kt;
+                    const int width = res ? p.rp : p.K;
+                    const int steps = min(4, (width - kk * BK) / 64);
+                    const int na = (steps + 1) / 2;
+                    const uint32_t a_base = smem_u32(sA + s * A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + s * B_BYTES);
+                    const uint32_t sfa_base = smem_u32(sSFA + s * SFA_BYTES);
+                    const uint32_t sfb_base = smem_u32(sSFB + s * SFB_BYTES);
+                    for (int j = 0; j < na; ++j) {
+                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFA + 4 * j, sdesc_sf_atom(sfa_base + 512 * j));
+                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFB + 8 * j, sdesc_sf_atom(sfb_base + 512 * j));
+                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFB + 8 * j + 4,
+                                                  sdesc_sf_atom(sfb_base + 1024 + 512 * j));
+                    }
+                    for (int st = 0; st < steps; ++st) {
+                        tc_mma_mxf4_pair(tmem + acc_col, sdesc_kmajor_sw128(a_base + 32 * st),
+                                         sdesc_kmajor_sw128(b_base + 32 * st), (st & 1) ? id_odd : id_even,
+                                         tmem + TMEM_SFA + 4 * (st >> 1), tmem + TMEM_SFB + 8 * (st >> 1),
+                                         (kt > 0 || st > 0) ? 1u : 0u);
+                    }
+                    tc_commit_pair_mc(&empty[s], 0x3);
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                tc_commit_pair_mc(&acc_full[b], 0x3);
+            }
+            // drain: every pair MMA has finished before tensor memory is freed
+            tc_commit_pair_mc(drain, 0x1);
+            mbar_wait(drain, 0, 0x233u);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue (both CTAs)
+        const int ew = warp - EPI_WARP0;
+        const int quad = warp & 3;
+        const int half = ew >> 2;
+        int it = 0;
+        for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++it) {
+            const int n_blk = tile % p.num_n_tiles;
+            const int m_pair = tile / p.num_n_tiles;
+            const int b = it & 1;
+            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[b], static_cast<uint32_t>((it >> 1) & 1), 0x331u))) break;
+            tc_fence_after();
+            const uint32_t base = b ? TMEM_ACC1 : TMEM_ACC0;
+            const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + base + 128u * half;
+            // the 32-column chunk of this warp holding the shared columns [232, 256), or -1
+            const int c_ovl = (b == 0 && half == 1) ? 3 : ((b == 1 && half == 0) ? 0 : -1);
+            uint32_t packed[64];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c == c_ovl) {  // warp-uniform
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(t_row + 32u * c, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                    tc_fence_before();
+                    mbar_arrive_cluster(ovl_empty, 0);
+                }
+            }
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                if (c == c_ovl) continue;
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(t_row + 32u * c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            }
+            tc_fence_before();
+            mbar_arrive_cluster(&acc_empty[b], 0);
+            const int row = m_pair * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
+            const int col0 = n_blk * BN + 128 * half;
+            if (row < p.M && col0 < p.N) {
+                uint4* out = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(row) * p.N + col0);
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    out[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    cluster_sync();  // the peer's remote arrivals and the pair MMAs are done
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc_pair(tmem, TMEM_COLS);
+}
+
+}  // namespace serq

@@ -20,6 +20,7 @@
 #include "gemm_mxfp4.cuh"
 #include "gemm_int4.cuh"
 #include "gemm_mxfp4_decode.cuh"
+#include "gemm_mxfp4_pair.cuh"
 
 using namespace serq;
 
@@ -67,6 +68,8 @@ struct DeviceInfo {
     bool smem_set_mx = false;
     bool smem_set_i4 = false;
     bool smem_set_mxd = false;
+    bool smem_set_mxp = false;
+    int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
 };
 
 // split-K ranges of the small-M kernel: about two CTAs per SM, at most
@@ -532,7 +535,54 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
     const int tiles = num_m * num_n;
     const int grid = tiles < info->sms ? tiles : info->sms;
 
-    if (w->fmt == SERQ_FMT_MXFP4) {
+    if (w->fmt == SERQ_FMT_MXFP4 && M > 128) {
+        // CTA-pair kernel: 256 x 256 tiles, B halves split across the pair
+        if (!info->smem_set_mxp) {
+            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           mxp::SMEM_BYTES));
+            cudaLaunchConfig_t qc = {};
+            qc.gridDim = dim3(info->sms, 1, 1);
+            qc.blockDim = dim3(mxp::THREADS, 1, 1);
+            qc.dynamicSmemBytes = mxp::SMEM_BYTES;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = 2;
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            qc.attrs = &attr;
+            qc.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, serq_linear_mxfp4_pair_kernel, &qc) != cudaSuccess || n < 1) {
+                cudaGetLastError();
+                n = info->sms / 2;
+            }
+            info->pair_clusters = n;
+            info->smem_set_mxp = true;
+        }
+        CUtensorMap tm_b128, tm_br128;
+        tm_b128 = w->tm_w128;
+        tm_br128 = w->tm_r128;
+        MxPairParams p;
+        p.M = M;
+        p.N = N;
+        p.K = K;
+        p.rp = rp;
+        p.num_n_tiles = (N + mxp::BN - 1) / mxp::BN;
+        p.num_tiles = p.num_n_tiles * ((M + 2 * mxp::BM - 1) / (2 * mxp::BM));
+        p.k_tiles_main = (K + mxp::BK - 1) / mxp::BK;
+        p.k_tiles_res = (rp + mxp::BK - 1) / mxp::BK;
+        p.atoms_k_main = K / 128;
+        p.atoms_k_res = (rp + 127) / 128;
+        p.row_blocks_a = (M + 127) / 128;
+        p.sfa = static_cast<const uint8_t*>(xs);
+        p.sfb = static_cast<const uint8_t*>(w->wsc);
+        p.sfa_r = static_cast<const uint8_t*>(xss);
+        p.sfb_r = static_cast<const uint8_t*>(w->rsc);
+        p.Y = static_cast<__nv_bfloat16*>(Y);
+        const int pairs = info->pair_clusters;
+        const int grid2 = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
+        serq_linear_mxfp4_pair_kernel<<<grid2, mxp::THREADS, mxp::SMEM_BYTES, cs>>>(tm_a, tm_b128, tm_ar, tm_br128, p);
+    } else if (w->fmt == SERQ_FMT_MXFP4) {
         if (!info->smem_set_mx) {
             SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                            mx::SMEM_BYTES));
