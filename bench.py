@@ -78,6 +78,12 @@ def barrier(pg):
             pg.barrier()
 
 
+def whole_job_tops(world: int, step_flops: float, ms_per_step: float) -> float:
+    """Aggregate throughput of `world` replicas that each ran one step of
+    `step_flops` in `ms_per_step` (the slowest rank's time)."""
+    return world * step_flops / (ms_per_step * 1e-3) / 1e12
+
+
 def max_over_ranks(pg, value: float) -> float:
     if pg is None:
         return value
@@ -223,7 +229,7 @@ def time_steps(layers, steps, warmup, pg, per_gemm=True, sampler=None):
     return total_ms, gemm_ms
 
 
-def time_e2e(layers, steps, warmup):
+def time_e2e(layers, steps, warmup, pg=None):
     """Same step through the public API with host buffers: pinned H2D of X^, D2H of Y, every step."""
     import torch
     import w4a4_post_quantization_serq_b200 as S
@@ -240,11 +246,14 @@ def time_e2e(layers, steps, warmup):
         step()
     torch.cuda.synchronize()
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(pg)
+    torch.cuda.synchronize()
     start.record()
     for _ in range(steps):
         step()
     end.record()
     torch.cuda.synchronize()
+    barrier(pg)
     S.serq_device_status()
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out)
@@ -420,9 +429,9 @@ def main():
     clocks = sampler.stop() if sampler is not None else None
     total_ms = max_over_ranks(pg, total_ms)
     ms_per_step = total_ms / args.steps
-    value = world * step_flops / (ms_per_step * 1e-3) / 1e12
+    value = whole_job_tops(world, step_flops, ms_per_step)
 
-    # dominant kernel: serq_linear_mxfp4_kernel; its largest launch (gate/up,
+    # dominant kernel: the CTA-pair MXFP4 linear; its largest launch (gate/up,
     # two thirds of the step's flops) is the roofline's unit
     peaks, peak_src = measured_peaks()
     fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
@@ -449,23 +458,22 @@ def main():
                        "l2": "inputs larger than L2 (a step touches ~300 MB)"},
             "roofline": roofline, "gpu_launches": 2 * len(layers) * args.steps, "clocks": clocks}
 
+    if not args.no_extras:
+        # end to end through the public API with host buffers, on every rank
+        e2e_ms, h2d, d2h = time_e2e(layers, max(3, args.steps // 4), 2, pg)
+        e2e_ms = max_over_ranks(pg, e2e_ms)
+        line["e2e"] = {"value": whole_job_tops(world, step_flops, e2e_ms), "unit": "TOPS",
+                       "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+    del layers
+    torch.cuda.empty_cache()
     if not args.no_extras and rank == 0:
         # SERQ overhead: the same step with r = 0 (plain W4A4)
-        del layers
-        torch.cuda.empty_cache()
         layers0 = build_layers(wl, r_override=0)
         t0, g0 = time_steps(layers0, args.steps, args.warmup, None)
         del layers0
         torch.cuda.empty_cache()
         line["overhead_vs_r0"] = {"ms_per_step_r0": t0 / args.steps, "step": ms_per_step / (t0 / args.steps) - 1,
                                   "serq_linear": sum(gemm_ms) / sum(g0) - 1}
-        # end to end through the public API with host buffers
-        layers = build_layers(wl)
-        e2e_ms, h2d, d2h = time_e2e(layers, max(3, args.steps // 4), 2)
-        line["e2e"] = {"value": step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS", "h2d_bytes_per_step": h2d,
-                       "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
-        del layers
-        torch.cuda.empty_cache()
         # INT4: LLaMA-2-7B q_proj shape
         wl2 = workload("qproj_int4")
         layers2 = build_layers(wl2)
