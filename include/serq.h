@@ -221,6 +221,21 @@ serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* 
  * (SERQ_ECUDA if the stream itself failed). */
 serq_status serq_device_status(serq_stream stream);
 
+/* ---------------------------------------------------------------------------
+ * serq_selftest_wait -- exercise the bounded pipeline wait (the pages have no
+ * counterpart; it exists so the timeout path can be tested on a GPU without
+ * stalling a real pipeline).
+ * One single-CTA kernel initialises an mbarrier expecting one arrival and
+ * waits for its first phase with the same bounded wait the GEMM pipelines use,
+ * but with a limit of `limit_cycles` SM clock cycles (1 .. 4e9). If `arrive`
+ * is non-zero the barrier is completed first and the wait returns at once;
+ * otherwise nothing completes it, the wait runs out after `limit_cycles`, and
+ * the kernel records site 0xF01 and returns: the next serq_device_status()
+ * reports SERQ_ETIMEOUT and clears the record. The CUDA context stays usable
+ * either way. Asynchronous on `stream`. Errors: EINVAL, ECUDA.
+ * ------------------------------------------------------------------------ */
+serq_status serq_selftest_wait(long long limit_cycles, int arrive, serq_stream stream);
+
 const char* serq_last_error(void); /* thread-local message of the last failure */
 const char* serq_version(void);
 

@@ -64,3 +64,9 @@ def test_prepare_rejects_bad_descriptors(lib):
 
 def test_linear_rejects_null_weight(lib):
     assert lib.serq_linear(None, 4, 16, 16, None, None, 16, None, None) == N.SERQ_EINVAL
+
+
+def test_selftest_wait_rejects_bad_limits(lib):
+    for bad in (0, -1, 4_000_000_001):
+        assert lib.serq_selftest_wait(bad, 1, None) == N.SERQ_EINVAL
+        assert b"limit_cycles" in lib.serq_last_error()

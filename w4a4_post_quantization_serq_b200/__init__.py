@@ -18,6 +18,7 @@ from .serq import (  # noqa: F401
     serq_linear_small_m_noalloc,
     serq_prepare,
     serq_quant_act,
+    serq_selftest_wait,
     serq_version,
     serq_weight_get_view,
 )

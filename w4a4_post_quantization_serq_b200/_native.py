@@ -49,6 +49,7 @@ _SIGNATURES = {
                             c_void_p]),
     "serq_linear_small_m_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "serq_selftest_wait": (c_int, [ctypes.c_longlong, c_int, c_void_p]),
     "serq_device_status": (c_int, [c_void_p]),
     "serq_last_error": (c_char_p, []),
     "serq_version": (c_char_p, []),

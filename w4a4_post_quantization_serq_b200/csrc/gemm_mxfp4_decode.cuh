@@ -8,10 +8,22 @@
 //    K-tiles ("量化推理": one extra r x N product, no intermediate
 //    quantization) are cut into S contiguous ranges; CTA (n_blk, split)
 //    streams 128 weight rows over its range;
-//  * each CTA writes fp32 partial sums to a workspace; the last CTA of an
-//    output block (ticket counter) adds the S partials in split order (a
-//    fixed order, so results do not depend on scheduling), writes bf16 Y and
-//    resets the counter for the next call.
+//  * split reduction, two forms (template flag):
+//    - cluster: the S split CTAs of an output block form one thread-block
+//      cluster (1 x S x 1); each parks its fp32 partial sums in its own
+//      shared memory, and after a cluster barrier CTA c adds, for its 1/S
+//      share of the block's outputs, the S partials read over distributed
+//      shared memory in split order, and writes bf16 Y. No workspace.
+//    - workspace: each CTA writes its partial sums to a global workspace; the
+//      last CTA of an output block (ticket counter) adds the S partials in
+//      split order, writes bf16 Y and resets the counter for the next call.
+//    Both add in split order from 0, so results do not depend on scheduling
+//    and the two forms agree bit for bit;
+//  * programmatic dependent launch: after its set-up each CTA lets the next
+//    kernel of the stream start, and the weight tiles of the first stages are
+//    requested before waiting for the preceding kernel; token data is read,
+//    and the workspace and Y are written, only after that wait. Weight
+//    streaming of consecutive linears thus overlaps the previous one's tail.
 #pragma once
 
 #include <cstdint>
@@ -37,7 +49,9 @@ constexpr uint32_t TMEM_COLS = 32;
 constexpr uint32_t TMEM_ACC = 0;                 // 16 fp32 columns (tokens)
 constexpr uint32_t TMEM_SFA = 16;                // 2 atoms x 4 columns
 constexpr uint32_t TMEM_SFB = 24;                // 2 atoms x 4 columns
-constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 1024 + 256;
+constexpr int PART_BYTES = MAX_TOKENS * BM * 4;  // this CTA's fp32 partial sums (cluster form)
+constexpr int MAX_SPLITS = 8;                    // portable cluster size
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + PART_BYTES + 1024 + 256;
 
 }  // namespace mxd
 
@@ -51,8 +65,8 @@ struct MxDecodeParams {
     const uint8_t* sf_x;    // token scale atoms (main)
     const uint8_t* sf_wr;   // residual scale atoms
     const uint8_t* sf_xr;   // salient-slice scale atoms
-    float* partial;         // [splits][M][N] workspace
-    unsigned int* tickets;  // [N / 128], zero between calls
+    float* partial;         // workspace form: [splits][M][N]
+    unsigned int* tickets;  // workspace form: [N / 128], zero between calls
     __nv_bfloat16* Y;
 };
 
@@ -66,6 +80,7 @@ __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&v)
         : "memory");
 }
 
+template <bool kClusterReduce>
 __global__ void __launch_bounds__(mxd::THREADS)
 serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                                 const __grid_constant__ CUtensorMap tm_wr, const __grid_constant__ CUtensorMap tm_xr,
@@ -77,7 +92,8 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     uint8_t* sB = sA + STAGES * A_BYTES;
     uint8_t* sSFA = sB + STAGES * B_BYTES;
     uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);
+    float* spart = reinterpret_cast<float*>(sSFB + STAGES * SFB_BYTES);  // [MAX_TOKENS][BM]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES + PART_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* drain = acc_full + 1;
@@ -108,24 +124,43 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    pdl_launch_dependents();
 
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            for (int kt = kt0; kt < kt1; ++kt) {
-                if (!mbar_wait(&empty[s], ph ^ 1u, 0x121u)) break;
+            // weights (independent of the preceding kernel) of the first stages first
+            const int pre = min(STAGES, kt1 - kt0);
+            for (int i = 0; i < pre; ++i) {
+                const int kt = kt0 + i;
                 const bool res = kt >= p.k_tiles_main;
                 const int kk = res ? kt - p.k_tiles_main : kt;
                 const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
                 const int na = min(2, atoms - 2 * kk);
-                mbar_arrive_expect_tx(&full[s], A_BYTES + p.n_tokens_mma * BK_BYTES + 2u * na * 512u);  // token box = n_tokens_mma rows
-                tma_load_2d(sA + s * A_BYTES, res ? &tm_wr : &tm_w, &full[s], kk * BK_BYTES, n_blk * BM);
-                tma_load_2d(sB + s * B_BYTES, res ? &tm_xr : &tm_x, &full[s], kk * BK_BYTES, 0);
-                bulk_load(sSFA + s * SFA_BYTES,
+                // token box = n_tokens_mma rows
+                mbar_arrive_expect_tx(&full[i], A_BYTES + p.n_tokens_mma * BK_BYTES + 2u * na * 512u);
+                tma_load_2d(sA + i * A_BYTES, res ? &tm_wr : &tm_w, &full[i], kk * BK_BYTES, n_blk * BM);
+                bulk_load(sSFA + i * SFA_BYTES,
                           (res ? p.sf_wr : p.sf_w) + (static_cast<size_t>(n_blk) * atoms + 2 * kk) * 512, na * 512,
-                          &full[s]);
+                          &full[i]);
+            }
+            pdl_wait_prerequisites();
+            int s = 0;
+            uint32_t ph = 0;
+            for (int kt = kt0; kt < kt1; ++kt) {
+                const bool res = kt >= p.k_tiles_main;
+                const int kk = res ? kt - p.k_tiles_main : kt;
+                const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
+                const int na = min(2, atoms - 2 * kk);
+                if (kt - kt0 >= pre) {
+                    if (!mbar_wait(&empty[s], ph ^ 1u, 0x121u)) break;
+                    mbar_arrive_expect_tx(&full[s], A_BYTES + p.n_tokens_mma * BK_BYTES + 2u * na * 512u);
+                    tma_load_2d(sA + s * A_BYTES, res ? &tm_wr : &tm_w, &full[s], kk * BK_BYTES, n_blk * BM);
+                    bulk_load(sSFA + s * SFA_BYTES,
+                              (res ? p.sf_wr : p.sf_w) + (static_cast<size_t>(n_blk) * atoms + 2 * kk) * 512,
+                              na * 512, &full[s]);
+                }
+                tma_load_2d(sB + s * B_BYTES, res ? &tm_xr : &tm_x, &full[s], kk * BK_BYTES, 0);
                 bulk_load(sSFB + s * SFB_BYTES, (res ? p.sf_xr : p.sf_x) + static_cast<size_t>(2 * kk) * 512,
                           na * 512, &full[s]);
                 if (++s == STAGES) {
@@ -190,38 +225,71 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
         // ------------------------------------------------------------ epilogue: partial sums
         const int quad = warp & 3;
         const int n = n_blk * BM + quad * 32 + lane;
+        pdl_wait_prerequisites();  // the preceding kernel is done with the workspace and Y
         if (__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, 0x321u))) {
             tc_fence_after();
             uint32_t v[16];
             tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TMEM_ACC, v);
             tmem_ld_wait();
-            float* part = p.partial + static_cast<size_t>(split) * p.M * p.N;
+            if constexpr (kClusterReduce) {
+                const int row = quad * 32 + lane;
 #pragma unroll
-            for (int m = 0; m < MAX_TOKENS; ++m)
-                if (m < p.M) part[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[m]);
+                for (int m = 0; m < MAX_TOKENS; ++m)
+                    if (m < p.M) spart[m * BM + row] = __uint_as_float(v[m]);
+            } else {
+                float* part = p.partial + static_cast<size_t>(split) * p.M * p.N;
+#pragma unroll
+                for (int m = 0; m < MAX_TOKENS; ++m)
+                    if (m < p.M) part[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[m]);
+            }
         }
         tc_fence_before();
     }
 
     // ---------------------------------------------------------------- split reduction
-    __threadfence();
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        const unsigned int ticket = atomicAdd(&p.tickets[n_blk], 1u);
-        s_is_last = (ticket == static_cast<unsigned int>(p.splits - 1)) ? 1u : 0u;
-    }
-    __syncthreads();
-    if (s_is_last) {
-        __threadfence();
-        for (int idx = threadIdx.x; idx < p.M * BM; idx += blockDim.x) {
-            const int m = idx / BM;
-            const int n = n_blk * BM + idx % BM;
+    pdl_wait_prerequisites();
+    if constexpr (kClusterReduce) {
+        __syncwarp();
+        cluster_sync();  // every split's partial sums are in its CTA's shared memory
+        const uint32_t rank = cluster_ctarank();  // == split: the cluster spans the S splits of this block
+        const int total = p.M * BM;
+        const int chunk = (total + p.splits - 1) / p.splits;
+        const int lo = static_cast<int>(rank) * chunk;
+        const int hi = min(total, lo + chunk);
+        const uint32_t local = smem_u32(spart);
+        for (int idx = lo + static_cast<int>(threadIdx.x); idx < hi; idx += blockDim.x) {
+            float part[MAX_SPLITS];
+#pragma unroll
+            for (int sp = 0; sp < MAX_SPLITS; ++sp)
+                part[sp] = sp < p.splits ? ld_shared_cluster_f32(mapa_shared(local + 4u * idx, sp)) : 0.0f;
             float acc = 0.0f;
-            for (int sp = 0; sp < p.splits; ++sp)
-                acc += __ldcg(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n);
-            p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc);
+#pragma unroll
+            for (int sp = 0; sp < MAX_SPLITS; ++sp)
+                if (sp < p.splits) acc += part[sp];
+            const int m = idx / BM;
+            p.Y[static_cast<size_t>(m) * p.N + n_blk * BM + idx % BM] = __float2bfloat16_rn(acc);
         }
-        if (threadIdx.x == 0) p.tickets[n_blk] = 0u;
+        cluster_sync();  // no CTA leaves while a peer still reads its partial sums
+    } else {
+        __threadfence();
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            const unsigned int ticket = atomicAdd(&p.tickets[n_blk], 1u);
+            s_is_last = (ticket == static_cast<unsigned int>(p.splits - 1)) ? 1u : 0u;
+        }
+        __syncthreads();
+        if (s_is_last) {
+            __threadfence();
+            for (int idx = threadIdx.x; idx < p.M * BM; idx += blockDim.x) {
+                const int m = idx / BM;
+                const int n = n_blk * BM + idx % BM;
+                float acc = 0.0f;
+                for (int sp = 0; sp < p.splits; ++sp)
+                    acc += __ldcg(p.partial + (static_cast<size_t>(sp) * p.M + m) * p.N + n);
+                p.Y[static_cast<size_t>(m) * p.N + n] = __float2bfloat16_rn(acc);
+            }
+            if (threadIdx.x == 0) p.tickets[n_blk] = 0u;
+        }
     }
 
     tc_fence_before();

@@ -104,6 +104,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
                       float* __restrict__ xs, uint32_t* __restrict__ xsq, float* __restrict__ xss) {
     __shared__ float red[64];
+    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
     const int m = blockIdx.x;
     const int nchunk = K >> 3;
     const uint4* row = X + static_cast<size_t>(m) * nchunk;
@@ -158,6 +159,7 @@ __global__ void __launch_bounds__(kQuantThreads)
 quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
                        uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
                        uint8_t* __restrict__ xss_atoms) {
+    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
     const int m = blockIdx.x;
     const int nchunk = K >> 3;
     const int atoms_k = (K / 32 + 3) / 4;

@@ -68,20 +68,37 @@ struct DeviceInfo {
     bool smem_set_mx = false;
     bool smem_set_i4 = false;
     bool smem_set_mxd = false;
+    int decode_slots = 0;   // co-resident small-M CTAs on the device (CTAs per SM x SMs)
     bool smem_set_mxp = false;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
 };
 
-// split-K ranges of the small-M kernel: about two CTAs per SM, at most
-// kMaxDecodeSplits, never more than the number of K-tiles
-constexpr int kMaxDecodeSplits = 8;
+// split-K ranges of the small-M kernel: as many as keep every CTA of the
+// launch co-resident (one wave over `slots` CTA slots), at most
+// kMaxDecodeSplits (the portable cluster size), never more than the K-tiles
+constexpr int kMaxDecodeSplits = mxd::MAX_SPLITS;
 constexpr int kMaxDecodeTokens = 16;
 
-int decode_splits(int n_blocks, int k_tiles, int sms) {
-    int s = (2 * sms + n_blocks - 1) / n_blocks;
+int decode_splits(int n_blocks, int k_tiles, int slots) {
+    int s = slots / n_blocks;
     if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
     if (s > k_tiles) s = k_tiles;
     return s < 1 ? 1 : s;
+}
+
+// One-time per-device set-up of both forms of the small-M kernel.
+serq_status decode_setup(DeviceInfo* info) {
+    if (info->smem_set_mxd) return SERQ_OK;
+    SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   mxd::SMEM_BYTES));
+    SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel<false>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, mxd::SMEM_BYTES));
+    int per_sm = 0;
+    SERQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, serq_linear_mxfp4_decode_kernel<true>,
+                                                            mxd::THREADS, mxd::SMEM_BYTES));
+    info->decode_slots = (per_sm < 1 ? 1 : per_sm) * info->sms;
+    info->smem_set_mxd = true;
+    return SERQ_OK;
 }
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -166,8 +183,6 @@ struct serq_weight {
     CUtensorMap tm_r;
     CUtensorMap tm_w128;   // A operand of the small-M kernel (128-row boxes, MXFP4)
     CUtensorMap tm_r128;
-    float* dec_partial;    // small-M split-K workspace [kMaxDecodeSplits][16][N] (MXFP4)
-    unsigned int* dec_tickets;  // [N / 128], zero between calls
 };
 
 // ============================================================== allocation-free small-M entry
@@ -196,6 +211,20 @@ serq_status noalloc_scratch(int dev, void** out) {
     return SERQ_OK;
 }
 }  // namespace
+
+// One bounded mbarrier wait, completed first or left to run out (site 0xF01).
+__global__ void wait_selftest_kernel(long long limit_cycles, int arrive) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (arrive) mbar_arrive(&bar);
+        mbar_wait_limit(&bar, 0u, 0xF01u, limit_cycles);
+    }
+}
 
 extern "C" {
 
@@ -294,9 +323,6 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     const size_t o_perm = take(4u * K), o_s = take(4u * K), o_sp = take(4u * K), o_inv = take(4u * K);
     const size_t o_wq = take(w->wq_bytes), o_wsc = take(w->wsc_bytes);
     const size_t o_rq = take(w->rq_bytes), o_rsc = take(w->rsc_bytes);
-    const bool mx = fmt == SERQ_FMT_MXFP4;
-    const size_t o_dp = take(mx ? sizeof(float) * kMaxDecodeSplits * kMaxDecodeTokens * static_cast<size_t>(N) : 0);
-    const size_t o_dt = take(mx ? 4u * (N / 128) : 0);
     const size_t keep = off;
     const size_t o_b = take(4u * K), o_col = take(4u * N);
     void* arena = nullptr;
@@ -317,8 +343,6 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     w->wsc = base + o_wsc;
     w->rq = base + o_rq;
     w->rsc = base + o_rsc;
-    w->dec_partial = mx ? reinterpret_cast<float*>(base + o_dp) : nullptr;
-    w->dec_tickets = mx ? reinterpret_cast<unsigned int*>(base + o_dt) : nullptr;
     float* tmp_b = reinterpret_cast<float*>(base + o_b);
     unsigned int* tmp_col = reinterpret_cast<unsigned int*>(base + o_col);
 
@@ -376,7 +400,7 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     } else {
         w->tm_r = w->tm_w;
     }
-    if (mx) {
+    if (fmt == SERQ_FMT_MXFP4) {
         if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return bail(st);
         if (rp > 0) {
             if (serq_status st = make_map(&w->tm_r128, w->rq, rp / 2, N, 128, 128, true)) return bail(st);
@@ -490,11 +514,7 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         } else {
             tm_xr = tm_x;
         }
-        if (!info->smem_set_mxd) {
-            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, mxd::SMEM_BYTES));
-            info->smem_set_mxd = true;
-        }
+        if (serq_status st = decode_setup(info)) return st;
         MxDecodeParams p;
         p.M = M;
         p.N = N;
@@ -504,20 +524,34 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
         p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
         const int n_blocks = N / mxd::BM;
-        p.splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
+        p.splits = decode_splits(n_blocks, p.k_tiles_total, info->decode_slots);
         p.atoms_k_main = K / 128;
         p.atoms_k_res = (rp + 127) / 128;
         p.sf_w = static_cast<const uint8_t*>(w->wsc);
         p.sf_x = static_cast<const uint8_t*>(xs);
         p.sf_wr = static_cast<const uint8_t*>(w->rsc);
         p.sf_xr = static_cast<const uint8_t*>(xss);
-        p.partial = w->dec_partial;
-        p.tickets = w->dec_tickets;
+        p.partial = nullptr;  // cluster form: partial sums stay in shared memory
+        p.tickets = nullptr;
         p.Y = static_cast<__nv_bfloat16*>(Y);
-        const dim3 grid(n_blocks, p.splits);
-        serq_linear_mxfp4_decode_kernel<<<grid, mxd::THREADS, mxd::SMEM_BYTES, cs>>>(w->tm_w128, tm_x, w->tm_r128,
-                                                                                      tm_xr, p);
-        SERQ_CUDA(cudaGetLastError());
+        // the S splits of an output block form one cluster; programmatic dependent
+        // launch lets the weight stream start under the preceding kernel's tail
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(n_blocks, p.splits, 1);
+        cfg.blockDim = dim3(mxd::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = mxd::SMEM_BYTES;
+        cfg.stream = cs;
+        cudaLaunchAttribute attr[2];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = static_cast<unsigned>(p.splits);
+        attr[0].val.clusterDim.z = 1;
+        attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[1].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 2;
+        SERQ_CUDA(cudaLaunchKernelEx(&cfg, serq_linear_mxfp4_decode_kernel<true>, w->tm_w128, tm_x, w->tm_r128, tm_xr,
+                                     p));
         return SERQ_OK;
     }
 
@@ -671,11 +705,7 @@ serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* 
         tm_wr = tm_w;
         tm_xr = tm_x;
     }
-    if (!info->smem_set_mxd) {
-        SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       mxd::SMEM_BYTES));
-        info->smem_set_mxd = true;
-    }
+    if (serq_status st = decode_setup(info)) return st;
     MxDecodeParams p;
     p.M = M;
     p.N = N;
@@ -685,7 +715,7 @@ serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* 
     p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
     p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
     const int n_blocks = N / mxd::BM;
-    int splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
+    int splits = decode_splits(n_blocks, p.k_tiles_total, info->decode_slots);
     while (splits > 1 && static_cast<size_t>(splits) * M * N > cap_floats) --splits;
     p.splits = splits;
     p.atoms_k_main = K / 128;
@@ -699,8 +729,17 @@ serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* 
     p.Y = static_cast<__nv_bfloat16*>(Y);
     // the array keeps the previous call's contents: the tickets must start at zero
     SERQ_CUDA(cudaMemsetAsync(p.tickets, 0, static_cast<size_t>(n_blocks) * sizeof(unsigned int), cs));
-    serq_linear_mxfp4_decode_kernel<<<dim3(n_blocks, splits), mxd::THREADS, mxd::SMEM_BYTES, cs>>>(tm_w, tm_x, tm_wr,
-                                                                                                  tm_xr, p);
+    serq_linear_mxfp4_decode_kernel<false><<<dim3(n_blocks, splits), mxd::THREADS, mxd::SMEM_BYTES, cs>>>(
+        tm_w, tm_x, tm_wr, tm_xr, p);
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
+serq_status serq_selftest_wait(long long limit_cycles, int arrive, serq_stream stream) {
+    if (limit_cycles < 1 || limit_cycles > 4000000000LL)
+        return fail(SERQ_EINVAL, "limit_cycles=%lld outside 1..4e9", limit_cycles);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    wait_selftest_kernel<<<1, 32, 0, cs>>>(limit_cycles, arrive != 0 ? 1 : 0);
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
 }

@@ -184,5 +184,10 @@ def serq_device_status(stream=None) -> None:
     N.check(N.load().serq_device_status(_stream(stream)))
 
 
+def serq_selftest_wait(limit_cycles: int, arrive: bool, stream=None) -> None:
+    """Launch the bounded-wait self-test kernel (see include/serq.h)."""
+    N.check(N.load().serq_selftest_wait(int(limit_cycles), 1 if arrive else 0, _stream(stream)))
+
+
 def serq_version() -> str:
     return N.load().serq_version().decode()
