@@ -39,8 +39,7 @@ def _full(lin, M, rows_sample):
     acc = torch.zeros(2, M, lin.N, dtype=torch.int32, device="cuda") if lin.fmt == "int4" else None
     Y = S.serq_linear(w, qa, acc_dbg=acc)
     S.serq_device_status()
-    res = {"xq": qa.xq.cpu().numpy(), "xs": qa.xs.cpu().numpy(),
-           "xsq": qa.xsq.cpu().numpy(), "xss": qa.xss.cpu().numpy()}
+    res = {k: (None if getattr(qa, k) is None else getattr(qa, k).cpu().numpy()) for k in ("xq", "xs", "xsq", "xss")}
     view = {k: v.cpu().numpy() for k, v in w.view().items()}
     # oracle
     a_o = O.calib_absmax(Xc)
@@ -82,3 +81,20 @@ def test_decode_mxfp4_full(name, M):
     wl = workload("decode_mxfp4")
     lin = [l for l in wl.linears if l.name == name][0]
     _full(lin, M, M)
+
+
+# The 32-block LLaMA-3-8B-shaped stack with its rank sweep r in {0, 16, 128,
+# 256}: every swept r on the first block's qkv, the ends of the sweep on the
+# other shapes (gate/up at r = 128 is the MLP case above), and two of the last
+# block's linears (other seeds).
+_STACK_CASES = ([(0, "qkv", r) for r in (0, 16, 128, 256)]
+                + [(0, "o", 16), (0, "o", 256), (0, "gate_up", 256), (0, "down", 16), (0, "down", 256)]
+                + [(31, "qkv", 128), (31, "o", 128)])
+
+
+@pytest.mark.parametrize("blk,name,r", _STACK_CASES)
+def test_stack_mxfp4_full(blk, name, r):
+    wl = workload("stack_mxfp4", r=r)
+    lin = [l for l in wl.linears if l.name == f"b{blk}.{name}"][0]
+    assert lin.r == r
+    _full(lin, wl.M, SAMPLE_ROWS)

@@ -39,7 +39,7 @@ constexpr int BM = 128;                 // output channels per CTA
 constexpr int BK = 256;                 // codes per K-tile
 constexpr int BK_BYTES = 128;
 constexpr int MAX_TOKENS = 16;
-constexpr int STAGES = 4;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK_BYTES;           // 16 KB weight codes
 constexpr int B_BYTES = MAX_TOKENS * BK_BYTES;   // 2 KB token codes
 constexpr int SFA_BYTES = 2 * 512;               // weight scale atoms
@@ -252,22 +252,32 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
         __syncwarp();
         cluster_sync();  // every split's partial sums are in its CTA's shared memory
         const uint32_t rank = cluster_ctarank();  // == split: the cluster spans the S splits of this block
-        const int total = p.M * BM;
+        const int total = p.M * (BM / 4);              // groups of 4 consecutive outputs
         const int chunk = (total + p.splits - 1) / p.splits;
         const int lo = static_cast<int>(rank) * chunk;
         const int hi = min(total, lo + chunk);
         const uint32_t local = smem_u32(spart);
-        for (int idx = lo + static_cast<int>(threadIdx.x); idx < hi; idx += blockDim.x) {
-            float part[MAX_SPLITS];
+        for (int g = lo + static_cast<int>(threadIdx.x); g < hi; g += blockDim.x) {
+            float4 part[MAX_SPLITS];
 #pragma unroll
             for (int sp = 0; sp < MAX_SPLITS; ++sp)
-                part[sp] = sp < p.splits ? ld_shared_cluster_f32(mapa_shared(local + 4u * idx, sp)) : 0.0f;
-            float acc = 0.0f;
+                if (sp < p.splits) part[sp] = ld_shared_cluster_v4f32(mapa_shared(local + 16u * g, sp));
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
 #pragma unroll
-            for (int sp = 0; sp < MAX_SPLITS; ++sp)
-                if (sp < p.splits) acc += part[sp];
-            const int m = idx / BM;
-            p.Y[static_cast<size_t>(m) * p.N + n_blk * BM + idx % BM] = __float2bfloat16_rn(acc);
+            for (int sp = 0; sp < MAX_SPLITS; ++sp) {
+                if (sp < p.splits) {
+                    acc.x += part[sp].x;
+                    acc.y += part[sp].y;
+                    acc.z += part[sp].z;
+                    acc.w += part[sp].w;
+                }
+            }
+            const int m = g / (BM / 4);
+            const int n = n_blk * BM + (g % (BM / 4)) * 4;
+            uint2 out;
+            out.x = pack_bf16x2(acc.x, acc.y);
+            out.y = pack_bf16x2(acc.z, acc.w);
+            *reinterpret_cast<uint2*>(p.Y + static_cast<size_t>(m) * p.N + n) = out;
         }
         cluster_sync();  // no CTA leaves while a peer still reads its partial sums
     } else {

@@ -10,8 +10,20 @@
 // plus TMA fits the shared-memory port, and six stages fit.
 //
 // Warp roles (each CTA): 0 TMA producer; 1 TMEM owner (+ MMA issuer in the
-// even CTA); 2 bridge (waits this CTA's stage, arrives on the even CTA's
-// "ready" barrier); 3..10 epilogue (tcgen05.ld -> release -> bf16 -> store).
+// even CTA); 2 idle; 3..10 epilogue (tcgen05.ld -> release -> bf16 -> store).
+//
+// Loads: codes and scale atoms all arrive by TMA tile loads (scale atoms as
+// rows of 256 B, two atoms per box). Both CTAs' loads of a stage count their
+// bytes on the even CTA's "full" barrier (.cta_group::2), which the even
+// CTA's producer arms with the bytes of both; the MMA issuer waits on that one
+// barrier, so a stage is handed over in a single hop.
+//
+// Epilogue stores: a thread holds one output row, so storing straight from
+// registers would make every warp store touch 32 rows with 16 B each (half
+// sectors, 32 L2 requests per instruction). Instead the two warps of a lane
+// quadrant take turns passing 64-column slices through a shared 4 KB tile
+// (swizzled, conflict-free) and store them eight threads per row: four full
+// 128 B lines per instruction.
 //
 // Two accumulators alternate between tiles so the epilogue of one tile
 // overlaps the MMAs of the next. Two 256-column fp32 tiles and the scale
@@ -41,6 +53,7 @@ constexpr int A_BYTES = BM * BK_BYTES;        // 16 KB
 constexpr int B_BYTES = BN_HALF * BK_BYTES;   // 16 KB
 constexpr int SFA_BYTES = 2 * 512;            // own 128 rows x 8 scales
 constexpr int SFB_BYTES = 4 * 512;            // all 256 rows x 8 scales
+constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // bytes one CTA loads per stage
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 3;
 constexpr int THREADS = (EPI_WARP0 + NUM_EPI_WARPS) * 32;
@@ -50,7 +63,9 @@ constexpr uint32_t TMEM_ACC1 = 232;           // shares columns [232, 256) with 
 constexpr uint32_t OVL_LO = 232;              // first shared column
 constexpr uint32_t TMEM_SFA = 488;
 constexpr uint32_t TMEM_SFB = 496;
-constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 1024 + 256;
+constexpr int STAGE_OUT_BYTES = 32 * 128;     // per lane quadrant: 32 rows x 64 bf16
+// the dynamic shared memory is declared 1024-byte aligned (128 B swizzle), so no pad
+constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + 4 * STAGE_OUT_BYTES + 256;
 
 }  // namespace mxp
 
@@ -59,28 +74,33 @@ struct MxPairParams {
     int num_n_tiles, num_tiles;     // pair tiles, n fastest
     int k_tiles_main, k_tiles_res;
     int atoms_k_main, atoms_k_res;
-    int row_blocks_a;               // ceil(M / 128): activation scale atoms that exist
-    const uint8_t* sfa;
-    const uint8_t* sfb;
-    const uint8_t* sfa_r;
-    const uint8_t* sfb_r;
     __nv_bfloat16* Y;
+};
+
+// Scale-atom tensor maps: the atom array viewed as rows of 256 B, box 256 x 4
+// (two 512 B atoms); rows past the end read as zeros.
+struct MxPairScaleMaps {
+    CUtensorMap sfa, sfb, sfa_r, sfb_r;
 };
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mxp::THREADS, 1)
 serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                               const __grid_constant__ CUtensorMap tm_ar, const __grid_constant__ CUtensorMap tm_br,
-                              const MxPairParams p) {
+                              const __grid_constant__ MxPairScaleMaps sf, const MxPairParams p) {
     using namespace mxp;
-    extern __shared__ uint8_t smem_raw[];
-    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    extern __shared__ __align__(1024) uint8_t smem_pair[];
+    uint8_t* smem = smem_pair;
+    if ((smem_u32(smem) & 1023u) != 0) {  // same in both CTAs of the pair: neither reaches a cluster barrier
+        if (threadIdx.x == 0) record_timeout(0x1A1u);
+        return;
+    }
     uint8_t* sA = smem;
     uint8_t* sB = sA + STAGES * A_BYTES;
     uint8_t* sSFA = sB + STAGES * B_BYTES;
     uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-    uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES);  // this CTA's loads landed
-    uint64_t* ready = full + STAGES;      // even CTA: both CTAs' loads landed
-    uint64_t* empty = ready + STAGES;     // stage consumed (multicast commit)
+    uint8_t* sOut = sSFB + STAGES * SFB_BYTES;                                // epilogue store tiles
+    uint64_t* full = reinterpret_cast<uint64_t*>(sOut + 4 * STAGE_OUT_BYTES);  // even CTA: both CTAs' loads landed
+    uint64_t* empty = full + STAGES;      // stage consumed (multicast commit)
     uint64_t* acc_full = empty + STAGES;  // [2] accumulator complete (multicast commit)
     uint64_t* acc_empty = acc_full + 2;   // [2] even CTA: both epilogues drained the accumulator
     uint64_t* ovl_empty = acc_empty + 2;  // even CTA: both epilogues drained the shared columns
@@ -97,7 +117,6 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&ready[s], 2);
             mbar_init(&empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -109,9 +128,13 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
         fence_mbar_init();
         tma_prefetch_desc(&tm_a);
         tma_prefetch_desc(&tm_b);
+        tma_prefetch_desc(&sf.sfa);
+        tma_prefetch_desc(&sf.sfb);
         if (p.k_tiles_res > 0) {
             tma_prefetch_desc(&tm_ar);
             tma_prefetch_desc(&tm_br);
+            tma_prefetch_desc(&sf.sfa_r);
+            tma_prefetch_desc(&sf.sfb_r);
         }
     }
     cluster_sync();
@@ -128,6 +151,7 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
     if (warp == 0) {
         // ------------------------------------------------------------ producer (both CTAs)
         if (lane == 0) {
+            const uint32_t full0 = mapa_shared(smem_u32(&full[0]), 0);  // the even CTA's barriers
             int s = 0;
             uint32_t ph = 0;
             bool ok = true;
@@ -135,8 +159,6 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                 const int n_blk = tile % p.num_n_tiles;
                 const int m_pair = tile / p.num_n_tiles;
                 const int a_rowblk = 2 * m_pair + static_cast<int>(rank);
-                const bool a_sf = a_rowblk < p.row_blocks_a;
-                const bool hi_half = (n_blk * BN + 128) < p.N;
                 for (int kt = 0; kt < total_k; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, 0x131u)) {
                         ok = false;
@@ -145,23 +167,18 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                     const bool res = kt >= p.k_tiles_main;
                     const int kk = res ? kt - p.k_tiles_main : kt;
                     const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
-                    const int na = min(2, atoms - 2 * kk);
-                    const uint8_t* sfa_src = res ? p.sfa_r : p.sfa;
-                    const uint8_t* sfb_src = res ? p.sfb_r : p.sfb;
-                    const uint32_t sf_bytes = static_cast<uint32_t>(na * 512) * ((a_sf ? 1u : 0u) + (hi_half ? 2u : 1u));
-                    mbar_arrive_expect_tx(&full[s], A_BYTES + B_BYTES + sf_bytes);
-                    tma_load_2d(sA + s * A_BYTES, res ? &tm_ar : &tm_a, &full[s], kk * BK_BYTES, a_rowblk * BM);
-                    tma_load_2d(sB + s * B_BYTES, res ? &tm_br : &tm_b, &full[s], kk * BK_BYTES,
-                                n_blk * BN + static_cast<int>(rank) * BN_HALF);
-                    if (a_sf)
-                        bulk_load(sSFA + s * SFA_BYTES,
-                                  sfa_src + (static_cast<size_t>(a_rowblk) * atoms + 2 * kk) * 512, na * 512, &full[s]);
-                    bulk_load(sSFB + s * SFB_BYTES,
-                              sfb_src + (static_cast<size_t>(2 * n_blk) * atoms + 2 * kk) * 512, na * 512, &full[s]);
-                    if (hi_half)
-                        bulk_load(sSFB + s * SFB_BYTES + 1024,
-                                  sfb_src + (static_cast<size_t>(2 * n_blk + 1) * atoms + 2 * kk) * 512, na * 512,
-                                  &full[s]);
+                    if (leader) mbar_arrive_expect_tx(&full[s], 2u * STAGE_TX);
+                    const uint32_t bar = full0 + 8u * static_cast<uint32_t>(s);
+                    tma_load_2d_pair(sA + s * A_BYTES, res ? &tm_ar : &tm_a, bar, kk * BK_BYTES, a_rowblk * BM);
+                    tma_load_2d_pair(sB + s * B_BYTES, res ? &tm_br : &tm_b, bar, kk * BK_BYTES,
+                                     n_blk * BN + static_cast<int>(rank) * BN_HALF);
+                    // scale atoms (2 per K-tile) as rows of 256 B
+                    tma_load_2d_pair(sSFA + s * SFA_BYTES, res ? &sf.sfa_r : &sf.sfa, bar, 0,
+                                     (a_rowblk * atoms + 2 * kk) * 2);
+                    tma_load_2d_pair(sSFB + s * SFB_BYTES, res ? &sf.sfb_r : &sf.sfb, bar, 0,
+                                     (2 * n_blk * atoms + 2 * kk) * 2);
+                    tma_load_2d_pair(sSFB + s * SFB_BYTES + 1024, res ? &sf.sfb_r : &sf.sfb, bar, 0,
+                                     ((2 * n_blk + 1) * atoms + 2 * kk) * 2);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -173,26 +190,6 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                 if (++s == STAGES) {
                     s = 0;
                     ph ^= 1u;
-                }
-            }
-        }
-    } else if (warp == 2) {
-        // ------------------------------------------------------------ bridge (both CTAs)
-        if (lane == 0) {
-            int s = 0;
-            uint32_t ph = 0;
-            bool ok = true;
-            for (int tile = cluster; tile < p.num_tiles && ok; tile += num_clusters) {
-                for (int kt = 0; kt < total_k; ++kt) {
-                    if (!mbar_wait(&full[s], ph, 0x133u)) {
-                        ok = false;
-                        break;
-                    }
-                    mbar_arrive_cluster(&ready[s], 0);
-                    if (++s == STAGES) {
-                        s = 0;
-                        ph ^= 1u;
-                    }
                 }
             }
         }
@@ -216,7 +213,7 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                 tc_fence_after();
                 const uint32_t acc_col = b ? TMEM_ACC1 : TMEM_ACC0;
                 for (int kt = 0; kt < total_k; ++kt) {
-                    if (!mbar_wait_cluster(&ready[s], ph, 0x232u)) {
+                    if (!mbar_wait_cluster(&full[s], ph, 0x232u)) {
                         ok = false;
                         break;
                     }
@@ -255,55 +252,85 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
             tc_commit_pair_mc(drain, 0x1);
             mbar_wait(drain, 0, 0x233u);
         }
-    } else {
+    } else if (warp >= EPI_WARP0) {
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int ew = warp - EPI_WARP0;
         const int quad = warp & 3;
         const int half = ew >> 2;
+        // the two warps of a lane quadrant (half 0 and half 1) share one 4 KB tile
+        const uint32_t out_tile = smem_u32(sOut + quad * STAGE_OUT_BYTES);
+        const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
         int it = 0;
         for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++it) {
             const int n_blk = tile % p.num_n_tiles;
             const int m_pair = tile / p.num_n_tiles;
             const int b = it & 1;
-            if (!__all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[b], static_cast<uint32_t>((it >> 1) & 1), 0x331u))) break;
-            tc_fence_after();
-            const uint32_t base = b ? TMEM_ACC1 : TMEM_ACC0;
-            const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + base + 128u * half;
-            // the 32-column chunk of this warp holding the shared columns [232, 256), or -1
-            const int c_ovl = (b == 0 && half == 1) ? 3 : ((b == 1 && half == 0) ? 0 : -1);
+            // on a timeout the warp skips the tile's work but keeps the tile-share barriers in step
+            const bool ok =
+                __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[b], static_cast<uint32_t>((it >> 1) & 1), 0x331u));
             uint32_t packed[64];
+            if (ok) {
+                tc_fence_after();
+                const uint32_t base = b ? TMEM_ACC1 : TMEM_ACC0;
+                const uint32_t t_row = tmem + (static_cast<uint32_t>(quad * 32) << 16) + base + 128u * half;
+                // the 32-column chunk of this warp holding the shared columns [232, 256), or -1
+                const int c_ovl = (b == 0 && half == 1) ? 3 : ((b == 1 && half == 0) ? 0 : -1);
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (c == c_ovl) {  // warp-uniform
+                for (int c = 0; c < 4; ++c) {
+                    if (c == c_ovl) {  // warp-uniform
+                        uint32_t v[32];
+                        tmem_ld_32x32b_x32(t_row + 32u * c, v);
+                        tmem_ld_wait();
+#pragma unroll
+                        for (int i = 0; i < 16; ++i)
+                            packed[c * 16 + i] =
+                                pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                        tc_fence_before();
+                        mbar_arrive_cluster(ovl_empty, 0);
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (c == c_ovl) continue;
                     uint32_t v[32];
                     tmem_ld_32x32b_x32(t_row + 32u * c, v);
                     tmem_ld_wait();
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                    tc_fence_before();
-                    mbar_arrive_cluster(ovl_empty, 0);
                 }
+                tc_fence_before();
+                mbar_arrive_cluster(&acc_empty[b], 0);
             }
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                if (c == c_ovl) continue;
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(t_row + 32u * c, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    packed[c * 16 + i] = pack_bf16x2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-            }
-            tc_fence_before();
-            mbar_arrive_cluster(&acc_empty[b], 0);
-            const int row = m_pair * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
+            const int row0 = m_pair * 2 * BM + static_cast<int>(rank) * BM + quad * 32;  // this warp's rows
             const int col0 = n_blk * BN + 128 * half;
-            if (row < p.M && col0 < p.N) {
-                uint4* out = reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(row) * p.N + col0);
+            // four rounds per tile over the shared tile: half 0's two 64-column slices,
+            // then half 1's. The owner writes its 32 rows x 128 B (16 B chunk c of row
+            // r at slot c ^ (r & 7): conflict-free), then stores them eight threads per
+            // row: 4 full 128 B lines per instruction.
 #pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    out[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            for (int round = 0; round < 4; ++round) {
+                if (ok && (round >> 1) == half && col0 < p.N) {  // warp-uniform
+                    const int cc = (round & 1) * 32;              // first packed word of the slice
+#pragma unroll
+                    for (int c = 0; c < 8; ++c)
+                        st_shared_v4(out_tile + static_cast<uint32_t>(lane) * 128u + ((static_cast<uint32_t>(c) ^ sw) << 4),
+                                     packed[cc + 4 * c], packed[cc + 4 * c + 1], packed[cc + 4 * c + 2],
+                                     packed[cc + 4 * c + 3]);
+                    __syncwarp();
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int r = i * 4 + (lane >> 3);
+                        const uint32_t slot = static_cast<uint32_t>(lane) & 7u;
+                        const uint4 v = ld_shared_v4(out_tile + static_cast<uint32_t>(r) * 128u + (slot << 4));
+                        const uint32_t c = slot ^ (static_cast<uint32_t>(r) & 7u);
+                        const int grow = row0 + r;
+                        if (grow < p.M)
+                            *reinterpret_cast<uint4*>(p.Y + static_cast<size_t>(grow) * p.N + col0 + (round & 1) * 64 +
+                                                      c * 8) = v;
+                    }
+                }
+                named_bar_sync(1 + quad, 64);  // the shared tile is free for the next round
             }
         }
     }

@@ -68,22 +68,28 @@ struct DeviceInfo {
     bool smem_set_mx = false;
     bool smem_set_i4 = false;
     bool smem_set_mxd = false;
-    int decode_slots = 0;   // co-resident small-M CTAs on the device (CTAs per SM x SMs)
     bool smem_set_mxp = false;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
 };
 
-// split-K ranges of the small-M kernel: as many as keep every CTA of the
-// launch co-resident (one wave over `slots` CTA slots), at most
-// kMaxDecodeSplits (the portable cluster size), never more than the K-tiles
+// split-K ranges of the small-M kernel. Two CTAs fit per SM. A launch first
+// takes one CTA per SM, leaving the other slot to the next launch, whose CTAs
+// then prefetch their weight stages while this one finishes; when a CTA
+// would still have more K-tiles than its ring holds, the launch takes both
+// slots instead (more bytes in flight). At most kMaxDecodeSplits (the
+// portable cluster size), never more than the K-tiles.
 constexpr int kMaxDecodeSplits = mxd::MAX_SPLITS;
 constexpr int kMaxDecodeTokens = 16;
 
-int decode_splits(int n_blocks, int k_tiles, int slots) {
-    int s = slots / n_blocks;
-    if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
-    if (s > k_tiles) s = k_tiles;
-    return s < 1 ? 1 : s;
+int decode_splits(int n_blocks, int k_tiles, int sms) {
+    auto fit = [&](int slots) {
+        int s = slots / n_blocks;
+        if (s > kMaxDecodeSplits) s = kMaxDecodeSplits;
+        if (s > k_tiles) s = k_tiles;
+        return s < 1 ? 1 : s;
+    };
+    const int s1 = fit(sms);
+    return (k_tiles + s1 - 1) / s1 > mxd::STAGES ? fit(2 * sms) : s1;
 }
 
 // One-time per-device set-up of both forms of the small-M kernel.
@@ -93,10 +99,11 @@ serq_status decode_setup(DeviceInfo* info) {
                                    mxd::SMEM_BYTES));
     SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel<false>,
                                    cudaFuncAttributeMaxDynamicSharedMemorySize, mxd::SMEM_BYTES));
-    int per_sm = 0;
-    SERQ_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, serq_linear_mxfp4_decode_kernel<true>,
-                                                            mxd::THREADS, mxd::SMEM_BYTES));
-    info->decode_slots = (per_sm < 1 ? 1 : per_sm) * info->sms;
+    // all of the unified L1/shared storage as shared memory, so that two CTAs fit per SM
+    SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel<true>,
+                                   cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
+    SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_decode_kernel<false>,
+                                   cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared));
     info->smem_set_mxd = true;
     return SERQ_OK;
 }
@@ -142,6 +149,15 @@ EncodeTiledFn encode_fn() {
 
 // 2-D uint8 tensor of `rows` rows of `inner` bytes; boxes of box_inner x box_rows.
 serq_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
+                     uint32_t box_rows, bool swizzle128);
+
+// MXFP4 scale-atom array (a multiple of 512 B) as rows of 256 B; a box is two
+// atoms (256 x 4). Rows past the end read as zeros.
+serq_status make_scale_map(CUtensorMap* map, const void* base, size_t bytes) {
+    return make_map(map, base, 256, bytes / 256, 256, 4, false);
+}
+
+serq_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
                      uint32_t box_rows, bool swizzle128) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return fail(SERQ_ECUDA, "cuTensorMapEncodeTiled is unavailable");
@@ -183,6 +199,8 @@ struct serq_weight {
     CUtensorMap tm_r;
     CUtensorMap tm_w128;   // A operand of the small-M kernel (128-row boxes, MXFP4)
     CUtensorMap tm_r128;
+    CUtensorMap tm_wsf;    // MXFP4 scale atoms as 256 B rows (box: two atoms)
+    CUtensorMap tm_rsf;
 };
 
 // ============================================================== allocation-free small-M entry
@@ -402,6 +420,12 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     }
     if (fmt == SERQ_FMT_MXFP4) {
         if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return bail(st);
+        if (serq_status st = make_scale_map(&w->tm_wsf, w->wsc, w->wsc_bytes)) return bail(st);
+        if (rp > 0) {
+            if (serq_status st = make_scale_map(&w->tm_rsf, w->rsc, w->rsc_bytes)) return bail(st);
+        } else {
+            w->tm_rsf = w->tm_wsf;
+        }
         if (rp > 0) {
             if (serq_status st = make_map(&w->tm_r128, w->rq, rp / 2, N, 128, 128, true)) return bail(st);
         } else {
@@ -524,7 +548,7 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
         p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
         const int n_blocks = N / mxd::BM;
-        p.splits = decode_splits(n_blocks, p.k_tiles_total, info->decode_slots);
+        p.splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
         p.atoms_k_main = K / 128;
         p.atoms_k_res = (rp + 127) / 128;
         p.sf_w = static_cast<const uint8_t*>(w->wsc);
@@ -607,15 +631,21 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.k_tiles_res = (rp + mxp::BK - 1) / mxp::BK;
         p.atoms_k_main = K / 128;
         p.atoms_k_res = (rp + 127) / 128;
-        p.row_blocks_a = (M + 127) / 128;
-        p.sfa = static_cast<const uint8_t*>(xs);
-        p.sfb = static_cast<const uint8_t*>(w->wsc);
-        p.sfa_r = static_cast<const uint8_t*>(xss);
-        p.sfb_r = static_cast<const uint8_t*>(w->rsc);
         p.Y = static_cast<__nv_bfloat16*>(Y);
+        const size_t row_blocks_a = static_cast<size_t>((M + 127) / 128);
+        MxPairScaleMaps sf;
+        if (serq_status st = make_scale_map(&sf.sfa, xs, row_blocks_a * p.atoms_k_main * 512)) return st;
+        sf.sfb = w->tm_wsf;
+        if (rp > 0) {
+            if (serq_status st = make_scale_map(&sf.sfa_r, xss, row_blocks_a * p.atoms_k_res * 512)) return st;
+        } else {
+            sf.sfa_r = sf.sfa;
+        }
+        sf.sfb_r = w->tm_rsf;
         const int pairs = info->pair_clusters;
         const int grid2 = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
-        serq_linear_mxfp4_pair_kernel<<<grid2, mxp::THREADS, mxp::SMEM_BYTES, cs>>>(tm_a, tm_b128, tm_ar, tm_br128, p);
+        serq_linear_mxfp4_pair_kernel<<<grid2, mxp::THREADS, mxp::SMEM_BYTES, cs>>>(tm_a, tm_b128, tm_ar, tm_br128,
+                                                                                    sf, p);
     } else if (w->fmt == SERQ_FMT_MXFP4) {
         if (!info->smem_set_mx) {
             SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -715,7 +745,7 @@ serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* 
     p.k_tiles_main = (K + mxd::BK - 1) / mxd::BK;
     p.k_tiles_total = p.k_tiles_main + (rp + mxd::BK - 1) / mxd::BK;
     const int n_blocks = N / mxd::BM;
-    int splits = decode_splits(n_blocks, p.k_tiles_total, info->decode_slots);
+    int splits = decode_splits(n_blocks, p.k_tiles_total, info->sms);
     while (splits > 1 && static_cast<size_t>(splits) * M * N > cap_floats) --splits;
     p.splits = splits;
     p.atoms_k_main = K / 128;
