@@ -316,6 +316,68 @@ def bench_decode(reps: int = 10, tokens=(1, 4, 16)):
     return out
 
 
+def bench_stack(ranks=(0, 16, 128, 256), reps: int = 3):
+    """The 32-block LLaMA-3-8B-shaped MXFP4 stack at M = 2048, per swept r.
+
+    Per block: qkv (4096 -> 6144), o (4096 -> 4096), gate/up (4096 -> 2x14336),
+    down (14336 -> 4096), each with its own prepared weight buffer (128
+    distinct buffers, ~3.7 GB at r = 128, so nothing stays in L2 between uses);
+    the block-0 weight and activation of each shape are prepared once and
+    copied into the 32 buffers (timing does not depend on the values).
+    Returns {r: {linears_ms, total_ms, TOPS_linears, TOPS_total}} where total
+    adds one serq_quant_act per linear input.
+    """
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import workload
+    out = {}
+    for r in ranks:
+        wl = workload("stack_mxfp4", r=r)
+        shapes = [l for l in wl.linears if l.name.startswith("b0.")]
+        blocks = len(wl.linears) // len(shapes)
+        per_shape = []
+        flops = 0.0
+        for lin in shapes:
+            W = torch.from_numpy(lin.W()).to(torch.bfloat16).cuda()
+            a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(wl.M)).to(torch.bfloat16).cuda())
+            pool = [S.serq_prepare(W, r, lin.fmt, act_absmax=a) for _ in range(blocks)]
+            del W
+            Xh = S.serq_fold_producer(pool[0], torch.from_numpy(lin.X(wl.M)).to(torch.bfloat16).cuda())
+            qa = S.serq_quant_act(Xh, r, lin.fmt)
+            Y = torch.empty(wl.M, lin.N, dtype=torch.bfloat16, device="cuda")
+            per_shape.append((lin, pool, Xh, qa, Y))
+            flops += blocks * 2.0 * wl.M * lin.N * (lin.K + r)
+
+        def run(with_quant):
+            for b in range(blocks):
+                for lin, pool, Xh, qa, Y in per_shape:
+                    if with_quant:
+                        S.serq_quant_act(Xh, r, lin.fmt, out=qa)
+                    S.serq_linear(pool[b], qa, Y=Y)
+
+        res = {}
+        for key, wq in (("linears_ms", False), ("total_ms", True)):
+            run(wq)
+            torch.cuda.synchronize()
+            start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            start.record()
+            for _ in range(reps):
+                run(wq)
+            end.record()
+            torch.cuda.synchronize()
+            S.serq_device_status()
+            res[key] = round(start.elapsed_time(end) / reps, 3)
+        res["TOPS_linears"] = round(flops / (res["linears_ms"] * 1e-3) / 1e12, 1)
+        res["TOPS_total"] = round(flops / (res["total_ms"] * 1e-3) / 1e12, 1)
+        out[f"r{r}"] = res
+        del per_shape
+        torch.cuda.empty_cache()
+    if "r0" in out:
+        for k, v in out.items():
+            v["overhead_vs_r0"] = round(v["total_ms"] / out["r0"]["total_ms"] - 1, 4)
+    return out
+
+
 # ----------------------------------------------------------------- CPU oracle
 def cpu_oracle_prepare(wl, r_override=None):
     """The oracle's offline preparation of every linear (not timed)."""
@@ -488,6 +550,7 @@ def main():
         line["decode"] = dec
         m16 = [v["M16"]["GBs"] for v in dec.values() if isinstance(v, dict) and "M16" in v]
         line["decode_GBs_M16_mean"] = sum(m16) / len(m16)
+        line["stack"] = bench_stack()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         secs, flops, cores = cpu_oracle_step(cpu_oracle_prepare(wl), args.cpu_rows)
         line["cpu_baseline"] = {"value": flops / secs / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
