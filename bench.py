@@ -45,6 +45,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (for profiler runs)")
     ap.add_argument("--only", default=None, help="time only the named linear of the workload (profiling)")
+    ap.add_argument("--profile-decode", default=None, metavar="SHAPE",
+                    help="run a few plain small-M launches of one decode shape (q, kv, gate_up, down) at "
+                         "--decode-m tokens and exit (for profilers)")
+    ap.add_argument("--decode-m", type=int, default=16)
     return ap.parse_args()
 
 
@@ -433,6 +437,24 @@ def captured_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
+def profile_decode(shape: str, M: int, launches: int = 4):
+    """A few plain launches of one decode-shape linear on separate weight copies
+    (no graph), so a profiler sees ordinary kernels that stream from HBM."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import workload
+    lin = [l for l in workload("decode_mxfp4").linears if l.name == shape][0]
+    W = torch.from_numpy(lin.W()).to(torch.bfloat16).cuda()
+    a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(16)).to(torch.bfloat16).cuda())
+    pool = [S.serq_prepare(W, lin.r, lin.fmt, act_absmax=a) for _ in range(launches)]
+    qa = S.serq_quant_act(S.serq_fold_producer(pool[0], torch.from_numpy(lin.X(M)).to(torch.bfloat16).cuda()),
+                          lin.r, lin.fmt)
+    for w in pool:
+        S.serq_linear(w, qa)
+    torch.cuda.synchronize()
+    S.serq_device_status()
+
+
 def reference_main(args, world, rank, pg):
     """The CPU oracle on a bounded token sample of the same workload (rank 0 only)."""
     from synth import workload
@@ -475,6 +497,9 @@ def main():
     import torch
     import w4a4_post_quantization_serq_b200 as S  # noqa: F401  (fails loudly without libserq.so)
     from synth import workload
+    if args.profile_decode:
+        profile_decode(args.profile_decode, args.decode_m)
+        return
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)

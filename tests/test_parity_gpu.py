@@ -102,6 +102,9 @@ def test_residual_reduces_error_on_gpu():
     (9, 768, 384, 0),         # r = 0, 16-token MMA with 7 padding tokens
     (16, 4096, 1024, 256),
     (16, 256, 128, 256),      # one K-tile each for main and residual
+    (3, 1152, 256, 64),       # odd scale-atom counts: a main K-tile and the residual K-tile with one atom each
+    (4, 32768, 256, 128),     # 129 K-tiles over 8 splits: ranges longer than a CTA's scale burst
+    (16, 14336, 384, 128),    # down-projection depth, 3 output blocks
 ])
 def test_decode_shapes(M, K, N, r):
     # small M takes the split-K streaming kernel (MXFP4)
