@@ -12,11 +12,19 @@
 // Warp roles (each CTA): 0 TMA producer; 1 TMEM owner (+ MMA issuer in the
 // even CTA); 2 idle; 3..10 epilogue (tcgen05.ld -> release -> bf16 -> store).
 //
-// Loads: codes and scale atoms all arrive by TMA tile loads (scale atoms as
-// rows of 256 B, two atoms per box). Both CTAs' loads of a stage count their
-// bytes on the even CTA's "full" barrier (.cta_group::2), which the even
-// CTA's producer arms with the bytes of both; the MMA issuer waits on that one
-// barrier, so a stage is handed over in a single hop.
+// Loads: codes and scale atoms all arrive by TMA tile loads. Both CTAs' loads
+// of a stage count their bytes on the even CTA's "full" barrier
+// (.cta_group::2), which the even CTA's producer arms with the bytes of both;
+// the MMA issuer waits on that one barrier, so a stage is handed over in a
+// single hop.
+//
+// Scale atoms reach tensor memory by tcgen05.cp, which the tensor pipe runs
+// in order with the MMAs: each copy costs pipe time between K-tiles, so the
+// weight scales come in a prepared "wide" layout (each 512 B atom repeated
+// four times, the two 128-row halves side by side, 4 KB per atom pair) that
+// one .128x256b copy moves per K-atom instead of two .32x128b.warpx4 copies.
+// The activation scales (written per call by serq_quant_act in the canonical
+// layout) keep the narrow copies: 4 copies per K-tile instead of 6.
 //
 // Epilogue stores: a thread holds one output row, so storing straight from
 // registers would make every warp store touch 32 rows with 16 B each (half
@@ -48,11 +56,11 @@ constexpr int BN = 256;                       // output channels per pair tile
 constexpr int BN_HALF = 128;                  // rows of B per CTA
 constexpr int BK_BYTES = 128;
 constexpr int BK = 256;
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_BYTES = BM * BK_BYTES;        // 16 KB
 constexpr int B_BYTES = BN_HALF * BK_BYTES;   // 16 KB
 constexpr int SFA_BYTES = 2 * 512;            // own 128 rows x 8 scales
-constexpr int SFB_BYTES = 4 * 512;            // all 256 rows x 8 scales
+constexpr int SFB_BYTES = 2 * 4096;           // all 256 rows x 8 scales, wide layout (2 atom pairs)
 constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // bytes one CTA loads per stage
 constexpr int NUM_EPI_WARPS = 8;
 constexpr int EPI_WARP0 = 3;
@@ -77,8 +85,9 @@ struct MxPairParams {
     __nv_bfloat16* Y;
 };
 
-// Scale-atom tensor maps: the atom array viewed as rows of 256 B, box 256 x 4
-// (two 512 B atoms); rows past the end read as zeros.
+// Scale tensor maps, arrays viewed as rows of 256 B (rows past the end read as
+// zeros): activation atoms with box 256 x 4 (two 512 B atoms), wide weight
+// scales with box 256 x 32 (two 4 KB atom pairs).
 struct MxPairScaleMaps {
     CUtensorMap sfa, sfb, sfa_r, sfb_r;
 };
@@ -176,9 +185,7 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                     tma_load_2d_pair(sSFA + s * SFA_BYTES, res ? &sf.sfa_r : &sf.sfa, bar, 0,
                                      (a_rowblk * atoms + 2 * kk) * 2);
                     tma_load_2d_pair(sSFB + s * SFB_BYTES, res ? &sf.sfb_r : &sf.sfb, bar, 0,
-                                     (2 * n_blk * atoms + 2 * kk) * 2);
-                    tma_load_2d_pair(sSFB + s * SFB_BYTES + 1024, res ? &sf.sfb_r : &sf.sfb, bar, 0,
-                                     ((2 * n_blk + 1) * atoms + 2 * kk) * 2);
+                                     (n_blk * atoms + 2 * kk) * 16);
                     if (++s == STAGES) {
                         s = 0;
                         ph ^= 1u;
@@ -229,9 +236,7 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                     const uint32_t sfb_base = smem_u32(sSFB + s * SFB_BYTES);
                     for (int j = 0; j < na; ++j) {
                         tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFA + 4 * j, sdesc_sf_atom(sfa_base + 512 * j));
-                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFB + 8 * j, sdesc_sf_atom(sfb_base + 512 * j));
-                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFB + 8 * j + 4,
-                                                  sdesc_sf_atom(sfb_base + 1024 + 512 * j));
+                        tc_cp_128x256b_pair(tmem + TMEM_SFB + 8 * j, sdesc_sf_wide(sfb_base + 4096 * j));
                     }
                     for (int st = 0; st < steps; ++st) {
                         tc_mma_mxf4_pair(tmem + acc_col, sdesc_kmajor_sw128(a_base + 32 * st),

@@ -259,4 +259,31 @@ __global__ void fold_producer_kernel(const __nv_bfloat16* __restrict__ src, int 
     dst[idx] = __float2bfloat16_rn(__fdiv_rn(x, s_perm[i]));
 }
 
+// Wide scale layout of the CTA-pair kernel: for each pair of 128-row blocks
+// (2p, 2p+1) and scale atom j, a 4 KB piece read by one tcgen05.cp .128x256b
+// as 128 rows x 32 bytes in 8-row x 16-byte core matrices (row group g at
+// 256 g, its two column halves 128 bytes apart). Row l must hold row l % 32 of
+// atom (2p, j) in its first half and of atom (2p+1, j) in its second, which is
+// what two .32x128b.warpx4 copies of the two atoms would put in the same 8
+// tensor-memory columns; so row group g, half h holds bytes [128 (g % 4),
+// +128) of atom (2p+h, j) (a missing odd block reads as zeros). One thread
+// per 16 bytes.
+__global__ void scale_widen_kernel(const uint8_t* __restrict__ atoms, int row_blocks, int atoms_k,
+                                   uint8_t* __restrict__ wide, size_t wide_bytes) {
+    const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;  // 16-byte unit
+    if (i * 16 >= wide_bytes) return;
+    const size_t piece = i / 256;                  // 4 KB pieces
+    const int within = static_cast<int>(i % 256);  // 16-byte units in the piece
+    const int group = within / 16;                 // 8-row group (256 bytes)
+    const int half = (within / 8) % 2;             // even / odd row block
+    const int row = within % 8;                    // row within the core matrix
+    const int j = static_cast<int>(piece % atoms_k);
+    const int pair = static_cast<int>(piece / atoms_k);
+    const int rb = 2 * pair + half;
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (rb < row_blocks)
+        v = reinterpret_cast<const uint4*>(atoms + (static_cast<size_t>(rb) * atoms_k + j) * 512)[8 * (group % 4) + row];
+    reinterpret_cast<uint4*>(wide)[i] = v;
+}
+
 }  // namespace serq

@@ -308,6 +308,12 @@ __device__ __forceinline__ void tc_cp_32x128b_warpx4_pair(uint32_t taddr, uint64
     asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
 }
 
+// Copy 128 rows x 32 bytes of shared memory into 128 tensor-memory lanes x 8
+// columns of both CTAs of the pair (each from its own shared memory).
+__device__ __forceinline__ void tc_cp_128x256b_pair(uint32_t taddr, uint64_t src_desc) {
+    asm volatile("tcgen05.cp.cta_group::2.128x256b [%0], %1;" ::"r"(taddr), "l"(src_desc) : "memory");
+}
+
 // Copy a 32-row x 16-byte block of shared memory into tensor memory, repeated
 // in all four 32-lane sub-partitions (the scale-factor feed of block-scaled MMA).
 __device__ __forceinline__ void tc_cp_32x128b_warpx4(uint32_t taddr, uint64_t src_desc) {
@@ -352,6 +358,18 @@ __device__ __forceinline__ uint64_t sdesc_sf_atom(uint32_t saddr) {
     uint64_t d = 0;
     d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
     d |= static_cast<uint64_t>(128 >> 4) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    return d;
+}
+
+// Descriptor of a 128-row x 32-byte unswizzled source in 8-row x 16-byte core
+// matrices: the two 16-byte column halves of a row group 128 bytes apart, row
+// groups 256 bytes apart (the 4 KB wide scale layout).
+__device__ __forceinline__ uint64_t sdesc_sf_wide(uint32_t saddr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+    d |= static_cast<uint64_t>(128 >> 4) << 16;   // leading byte offset: next 16-byte column half
+    d |= static_cast<uint64_t>(256 >> 4) << 32;   // stride byte offset: next 8-row group
     d |= static_cast<uint64_t>(1) << 46;
     return d;
 }

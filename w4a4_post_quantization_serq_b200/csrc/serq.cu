@@ -195,11 +195,15 @@ struct serq_weight {
     size_t rq_bytes;
     void* rsc;
     size_t rsc_bytes;
+    uint8_t* wscw;         // MXFP4 weight / residual scales in the wide layout of the CTA-pair kernel
+    size_t wscw_bytes;
+    uint8_t* rscw;
+    size_t rscw_bytes;
     CUtensorMap tm_w;      // B operand of the prefill kernels (256-row boxes)
     CUtensorMap tm_r;
     CUtensorMap tm_w128;   // A operand of the small-M kernel (128-row boxes, MXFP4)
     CUtensorMap tm_r128;
-    CUtensorMap tm_wsf;    // MXFP4 scale atoms as 256 B rows (box: two atoms)
+    CUtensorMap tm_wsf;    // wide MXFP4 scales as 256 B rows (box: two 4 KB atom pairs)
     CUtensorMap tm_rsf;
 };
 
@@ -330,6 +334,9 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     } else {
         w->wsc_bytes = atom_bytes(N, K / 32);
         w->rsc_bytes = rp > 0 ? atom_bytes(N, rp / 32) : 0;
+        const size_t pairs = static_cast<size_t>((N / 128 + 1) / 2);
+        w->wscw_bytes = pairs * (K / 128) * 4096;
+        w->rscw_bytes = rp > 0 ? pairs * ((rp + 127) / 128) * 4096 : 0;
     }
     // one arena: perm, s, s_perm, inv_s, wq, wsc, rq, rsc, then scratch
     size_t off = 0;
@@ -341,6 +348,7 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     const size_t o_perm = take(4u * K), o_s = take(4u * K), o_sp = take(4u * K), o_inv = take(4u * K);
     const size_t o_wq = take(w->wq_bytes), o_wsc = take(w->wsc_bytes);
     const size_t o_rq = take(w->rq_bytes), o_rsc = take(w->rsc_bytes);
+    const size_t o_wscw = take(w->wscw_bytes), o_rscw = take(w->rscw_bytes);
     const size_t keep = off;
     const size_t o_b = take(4u * K), o_col = take(4u * N);
     void* arena = nullptr;
@@ -361,6 +369,8 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     w->wsc = base + o_wsc;
     w->rq = base + o_rq;
     w->rsc = base + o_rsc;
+    w->wscw = base + o_wscw;
+    w->rscw = base + o_rscw;
     float* tmp_b = reinterpret_cast<float*>(base + o_b);
     unsigned int* tmp_col = reinterpret_cast<unsigned int*>(base + o_col);
 
@@ -406,6 +416,11 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
         if (r > 0)
             residual_mxfp4_kernel<<<dim3(N / 32, (rp / 32 + 7) / 8), qblock, 0, cs>>>(
                 W, w->perm, w->s_perm, K, N, r, rp, w->rq, static_cast<uint8_t*>(w->rsc));
+        scale_widen_kernel<<<static_cast<unsigned>((w->wscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
+            static_cast<const uint8_t*>(w->wsc), N / 128, K / 128, w->wscw, w->wscw_bytes);
+        if (rp > 0)
+            scale_widen_kernel<<<static_cast<unsigned>((w->rscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
+                static_cast<const uint8_t*>(w->rsc), N / 128, (rp + 127) / 128, w->rscw, w->rscw_bytes);
     }
     PREP_CUDA(cudaGetLastError());
     PREP_CUDA(cudaStreamSynchronize(cs));
@@ -420,9 +435,10 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     }
     if (fmt == SERQ_FMT_MXFP4) {
         if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return bail(st);
-        if (serq_status st = make_scale_map(&w->tm_wsf, w->wsc, w->wsc_bytes)) return bail(st);
+        if (serq_status st = make_map(&w->tm_wsf, w->wscw, 256, w->wscw_bytes / 256, 256, 32, false)) return bail(st);
         if (rp > 0) {
-            if (serq_status st = make_scale_map(&w->tm_rsf, w->rsc, w->rsc_bytes)) return bail(st);
+            if (serq_status st = make_map(&w->tm_rsf, w->rscw, 256, w->rscw_bytes / 256, 256, 32, false))
+                return bail(st);
         } else {
             w->tm_rsf = w->tm_wsf;
         }
