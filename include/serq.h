@@ -91,8 +91,10 @@ serq_status serq_calib_absmax(const void* X, int M, int K, float* absmax, serq_s
  * Inputs (device): W bf16 K x N; act_absmax fp32[K] or s fp32[K] (exactly one
  * non-NULL). Requirements: K % 128 == 0, N % 128 == 0, 0 <= r <= K.
  * On success *out owns device copies of perm, s, 1/s[perm], W^_q, Q(R) and
- * their scales. Synchronizes the stream. Errors: EINVAL, EUNSUPPORTED,
- * ENOMEM, ECUDA (nothing is leaked on failure).
+ * their scales (MXFP4: also a second, internal copy of both scale arrays in
+ * the layout the prefill kernel copies into tensor memory, 4x the scale
+ * bytes). Synchronizes the stream. Errors: EINVAL, EUNSUPPORTED, ENOMEM,
+ * ECUDA (nothing is leaked on failure).
  * ------------------------------------------------------------------------ */
 typedef struct {
     int K, N, r;
