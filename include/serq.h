@@ -173,6 +173,13 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
  * Inputs are serq_quant_act's outputs for the same (M, K, r, fmt).
  * Y: device bf16 [M][N]. acc_dbg: NULL, or (INT4 only) device int32
  * [2][M][N] receiving acc1 and acc2.
+ * Kernels (MXFP4): M <= 16 a split-K weight-streaming kernel (its split CTAs
+ * form a thread-block cluster; launched with programmatic dependent launch,
+ * so it may start streaming weights while the preceding kernel of the stream
+ * finishes, and reads xq/xs and writes Y only after it completes);
+ * 16 < M <= 128 a one-CTA tensor-core kernel; M > 128 a CTA-pair kernel.
+ * INT4: one tensor-core kernel for every M. Results do not depend on which
+ * kernel ran beyond fp32 summation order (MXFP4); INT4 accumulators are exact.
  * Errors: EINVAL (shape/format mismatch with w, NULL/unaligned pointers),
  * EUNSUPPORTED (not an sm_100 device).
  * ------------------------------------------------------------------------ */

@@ -79,7 +79,8 @@ constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) 
 
 struct MxPairParams {
     int M, N, K, rp;
-    int num_n_tiles, num_tiles;     // pair tiles, n fastest
+    int num_n_tiles, num_tiles;     // pair tiles, m fastest: the CTA pairs working at one time
+    int num_m_pairs;                // share weight tiles in L2 (tile = n_blk * num_m_pairs + m_pair)
     int k_tiles_main, k_tiles_res;
     int atoms_k_main, atoms_k_res;
     __nv_bfloat16* Y;
@@ -165,8 +166,8 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
             uint32_t ph = 0;
             bool ok = true;
             for (int tile = cluster; tile < p.num_tiles && ok; tile += num_clusters) {
-                const int n_blk = tile % p.num_n_tiles;
-                const int m_pair = tile / p.num_n_tiles;
+                const int n_blk = tile / p.num_m_pairs;
+                const int m_pair = tile % p.num_m_pairs;
                 const int a_rowblk = 2 * m_pair + static_cast<int>(rank);
                 for (int kt = 0; kt < total_k; ++kt) {
                     if (!mbar_wait(&empty[s], ph ^ 1u, 0x131u)) {
@@ -267,8 +268,8 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
         const uint32_t sw = static_cast<uint32_t>(lane) & 7u;
         int it = 0;
         for (int tile = cluster; tile < p.num_tiles; tile += num_clusters, ++it) {
-            const int n_blk = tile % p.num_n_tiles;
-            const int m_pair = tile / p.num_n_tiles;
+            const int n_blk = tile / p.num_m_pairs;
+            const int m_pair = tile % p.num_m_pairs;
             const int b = it & 1;
             // on a timeout the warp skips the tile's work but keeps the tile-share barriers in step
             const bool ok =

@@ -642,7 +642,8 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.K = K;
         p.rp = rp;
         p.num_n_tiles = (N + mxp::BN - 1) / mxp::BN;
-        p.num_tiles = p.num_n_tiles * ((M + 2 * mxp::BM - 1) / (2 * mxp::BM));
+        p.num_m_pairs = (M + 2 * mxp::BM - 1) / (2 * mxp::BM);
+        p.num_tiles = p.num_n_tiles * p.num_m_pairs;
         p.k_tiles_main = (K + mxp::BK - 1) / mxp::BK;
         p.k_tiles_res = (rp + mxp::BK - 1) / mxp::BK;
         p.atoms_k_main = K / 128;
