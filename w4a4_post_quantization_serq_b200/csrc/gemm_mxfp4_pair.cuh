@@ -5,9 +5,8 @@
 // CTA pair. Each CTA loads its own 128 rows of A and its own 128-row half of
 // B; one thread of the even CTA issues M = 256 MMAs that read both CTAs'
 // shared memory and write each CTA's 128 rows of D into that CTA's tensor
-// memory. Per CTA, a K-tile stage is 35 KB instead of the 51 KB of the
-// single-CTA 128 x 256 tile, so the shared-memory traffic of the tensor core
-// plus TMA fits the shared-memory port, and six stages fit.
+// memory. Per CTA a K-tile stage holds half the weight rows of the single-CTA
+// 128 x 256 tile (41 KB with the wide weight scales, 5 stages).
 //
 // Warp roles (each CTA): 0 TMA producer; 1 TMEM owner (+ MMA issuer in the
 // even CTA); 2 idle; 3..10 epilogue (tcgen05.ld -> release -> bf16 -> store).
