@@ -70,3 +70,33 @@ def test_selftest_wait_rejects_bad_limits(lib):
     for bad in (0, -1, 4_000_000_001):
         assert lib.serq_selftest_wait(bad, 1, None) == N.SERQ_EINVAL
         assert b"limit_cycles" in lib.serq_last_error()
+
+
+def test_calib_absmax_rejects_before_touching_device(lib):
+    assert lib.serq_calib_absmax(None, 4, 256, 16, None) == N.SERQ_EINVAL   # NULL X
+    assert lib.serq_calib_absmax(16, 0, 256, 16, None) == N.SERQ_EINVAL     # M < 1
+    assert lib.serq_calib_absmax(16, 4, 0, 16, None) == N.SERQ_EINVAL       # K < 1
+    assert lib.serq_calib_absmax(17, 4, 256, 16, None) == N.SERQ_EINVAL     # unaligned
+
+
+def test_view_and_fold_reject_null_weight(lib):
+    view = N.WeightView()
+    assert lib.serq_weight_get_view(None, ctypes.byref(view)) == N.SERQ_EINVAL
+    assert lib.serq_fold_producer(None, 16, 4, 32, None) == N.SERQ_EINVAL
+
+
+@pytest.mark.parametrize("M,K,Nn,r", [(0, 256, 256, 0), (17, 256, 256, 0), (4, 200, 256, 0), (4, 256, 200, 0),
+                                      (4, 65536, 256, 0), (4, 256, 256, 257), (4, 256, 256, -1)])
+def test_noalloc_rejects_bad_shapes(lib, M, K, Nn, r):
+    assert lib.serq_linear_small_m_noalloc(M, K, Nn, r, 16, 16, 16, 16, 16, 16, 16, 16, 16, None) == N.SERQ_EINVAL
+    assert lib.serq_last_error()
+
+
+def test_noalloc_rejects_null_and_unaligned(lib):
+    ok = (4, 256, 256, 16)
+    # NULL weight codes
+    assert lib.serq_linear_small_m_noalloc(*ok, None, 16, 16, 16, 16, 16, 16, 16, 16, None) == N.SERQ_EINVAL
+    # r > 0 without the residual / salient-slice buffers
+    assert lib.serq_linear_small_m_noalloc(*ok, 16, 16, None, 16, 16, 16, 16, 16, 16, None) == N.SERQ_EINVAL
+    # an unaligned output pointer
+    assert lib.serq_linear_small_m_noalloc(*ok, 16, 16, 16, 16, 16, 16, 16, 16, 24, None) == N.SERQ_EINVAL
