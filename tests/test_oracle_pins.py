@@ -393,3 +393,58 @@ def test_page_table_consistency():
     assert 2 ** (g["bits"] - 1) - 1 == g["int4_divisor"] == O.INT4_QMAX
     ppl = g["rank_ppl"]
     assert ppl["0"] > ppl["16"] > ppl["128"] > ppl["256"]
+
+
+# --------------------------------------------------------------------------
+# hand values for the helpers every parity test relies on: the bf16 storage
+# rounding of X^, the calibration maximum, the SAF divisor |W| and the
+# salient slice's own scale (tests/golden/oracle_hand_cases.json)
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", _golden("oracle_hand_cases.json")["bf16_rne"])
+def test_bf16_rne_hand_cases(case):
+    x = np.array([int(case["f32"], 16)], dtype=np.uint32).view(np.float32)
+    got = O.bf16_rne(x).view(np.uint32)[0]
+    assert got & 0xFFFF == 0
+    assert int(got >> 16) == int(case["bf16"], 16), case["why"]
+
+
+def test_calib_absmax_hand_values():
+    g = _golden("oracle_hand_cases.json")["calib_absmax"]
+    for xk, ak in (("X", "a"), ("X_square", "a_square")):
+        a = O.calib_absmax(np.array(g[xk], np.float32))
+        assert a.dtype == np.float32 and a.tolist() == g[ak]
+
+
+def test_saf_scales_use_weight_magnitude():
+    g = _golden("oracle_hand_cases.json")["saf_scales"]
+    s = O.saf_scales(np.array(g["a"], np.float32), np.array(g["W"], np.float32))
+    assert s.dtype == np.float32 and s.tolist() == g["s"], g["why"]
+
+
+def _row(case):
+    x = np.zeros((1, case["K"]), np.float32)
+    for c, v in case["x_nonzero"].items():
+        x[0, int(c)] = v
+    return x
+
+
+@pytest.mark.parametrize("case", _golden("oracle_hand_cases.json")["salient_slice"],
+                         ids=lambda c: f"{c['fmt']}-r{c['r']}")
+def test_salient_slice_hand_values(case):
+    x = _row(case)
+    qa = O.quant_act(x, case["r"], case["fmt"])
+    if case["fmt"] == "mxfp4":
+        assert qa.Ex[0].tolist() == case["E_main"]
+        assert qa.Exs[0].tolist() == case["E_slice"], case["why"]
+        assert qa.qxs.shape == (1, 32 * len(case["E_slice"]))
+    else:
+        assert float(qa.sx[0]) == case["scale_main"]
+        assert float(qa.sxs[0]) == case["scale_slice"], case["why"]
+        assert qa.qxs.shape == (1, case["r"])
+    for c, code in case["codes_main_first"].items():
+        assert int(qa.qx[0, int(c)]) == code, ("main", c)
+    expect = np.zeros(qa.qxs.shape[1], np.int64)
+    for c, code in case["codes_slice"].items():
+        expect[int(c)] = code
+    assert qa.qxs[0].astype(np.int64).tolist() == expect.tolist(), case["why"]
