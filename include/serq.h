@@ -61,7 +61,7 @@ typedef enum {
     SERQ_OK = 0,
     SERQ_EINVAL = 1,       /* bad argument: shape, pointer, alignment, format */
     SERQ_EUNSUPPORTED = 2, /* device is not sm_100 or shape outside the kernels' range */
-    SERQ_ENOMEM = 3,       /* device allocation failed (serq_prepare only) */
+    SERQ_ENOMEM = 3,       /* device allocation of a prepared weight failed */
     SERQ_ECUDA = 4,        /* a CUDA runtime call failed */
     SERQ_ETIMEOUT = 5      /* a kernel gave up waiting on a pipeline barrier */
 } serq_status;
@@ -131,6 +131,80 @@ typedef struct {
 } serq_weight_view;
 
 serq_status serq_weight_get_view(const serq_weight* w, serq_weight_view* out);
+
+/* ------------------------------------------------------------------------
+ * The prepared weight as an artefact: export, checkpoint and import.
+ *
+ * SERQ's offline stages produce the permuted, flattened and quantized linear
+ * once; at run time it costs nothing extra (reading notes Stage 3 and
+ * gist.science/zh 2.3: the permutation and 1/s are merged into the weights
+ * ahead of time). These calls move that artefact between processes and
+ * devices in a canonical host form:
+ *
+ *   perm     int32[K]           permuted position -> original channel
+ *   s        fp32[K]            SAF scales, original channel order (> 0)
+ *   inv_s    fp32[K]            1 / s[perm[i]] (IEEE division), permuted order
+ *   wq       u8[N][K/2]         packed W^_q (element 2j low nibble)
+ *   w_scale  INT4 : fp32[N]     per output channel
+ *            MXFP4: u8[N][K/32] E8M0 bytes, row-major (not the atom layout)
+ *   rq       u8[N][rp/2]        packed Q(R); codes at positions >= r are 0
+ *   r_scale  INT4 : fp32[N]     (zeros when r = 0)
+ *            MXFP4: u8[N][rp/32] E8M0, row-major; blocks past ceil(r/32) are 0
+ *
+ * rp = round_up(r, 64) (0 when r = 0). The caller owns every host buffer.
+ * ------------------------------------------------------------------------ */
+typedef struct {
+    int K, N, r, rp, fmt;
+    int32_t* perm;
+    float* s;
+    float* inv_s;
+    uint8_t* wq;
+    void* w_scale;
+    uint8_t* rq;
+    void* r_scale;
+} serq_weight_host;
+
+/* Copy a prepared weight into canonical host buffers. dst->K..fmt are set;
+ * each non-NULL pointer receives its part (NULL parts are skipped), so a
+ * first call with every pointer NULL just reports the shape. Synchronizes
+ * the weight's device. Errors: EINVAL (NULL w or dst), ECUDA. */
+serq_status serq_weight_export(const serq_weight* w, serq_weight_host* dst);
+
+/* Build a prepared weight on the current device from canonical host buffers
+ * (all non-NULL, except rq/r_scale when r = 0): for example one exported
+ * from another process, read from a checkpoint, or quantized by other
+ * tooling in this layout. The content is checked first: shape rules as for
+ * serq_prepare, rp = round_up(r, 64), perm a permutation of 0..K-1, s finite
+ * and > 0, inv_s[i] == 1/s[perm[i]] bit for bit, INT4 codes in [-7, 7] and
+ * scales finite and >= 0, no E8M0 byte 0xFF, zero codes / scale blocks past
+ * r. The result is bit-identical on export to the buffers it was built from.
+ * Synchronizes the stream. Errors: EINVAL (content), EUNSUPPORTED, ENOMEM,
+ * ECUDA; nothing is leaked on failure. */
+serq_status serq_weight_create_from_host(const serq_weight_host* src, serq_weight** out, serq_stream stream);
+
+/* Checkpoint file: a 64-byte header (magic "SERQWGT", version 1, fmt, K, N,
+ * r, rp, payload size, FNV-1a-64 checksum of the payload) followed by the
+ * canonical parts above in their listed order, little-endian.
+ *   serq_weight_save: export + write (synchronizes the weight's device).
+ *   serq_weight_load: read + check (header, size, checksum, content) +
+ *     serq_weight_create_from_host on the current device.
+ *   serq_weight_file_write / serq_weight_file_read: the same file from / to
+ *     host buffers, without a GPU. file_read sets dst->K..fmt and fills the
+ *     non-NULL pointers (a first call with every pointer NULL reports the
+ *     shape so the caller can size its buffers).
+ * Errors: EINVAL (NULL arguments, unreadable / unwritable / truncated /
+ * corrupt file, content), plus those of the device calls. */
+serq_status serq_weight_save(const serq_weight* w, const char* path);
+serq_status serq_weight_load(const char* path, serq_weight** out, serq_stream stream);
+serq_status serq_weight_file_write(const char* path, const serq_weight_host* src);
+serq_status serq_weight_file_read(const char* path, serq_weight_host* dst);
+
+/* Test hook (no counterpart in the paper): the next n device allocations of a
+ * prepared weight (serq_prepare, serq_weight_create_from_host,
+ * serq_weight_load) fail with SERQ_ENOMEM without calling cudaMalloc, so the
+ * out-of-memory path can be tested without exhausting the GPU. n = 0 clears
+ * it. Returns the previous count. */
+int serq_debug_fail_next_allocations(int n);
 
 /* ------------------------------------------------------------------------
  * Producer fold (Stage 3: "行/列排列离线合并到权重中"; gist.science/zh 2.3).

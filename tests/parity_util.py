@@ -128,3 +128,32 @@ def compare_y(Y_gpu: np.ndarray, Y_ref: np.ndarray, tol: float = YTOL):
     worst = float(rel.max(initial=0.0))
     assert worst <= tol, f"max row-normalised error {worst:.3e} > {tol}"
     return worst
+
+
+def oracle_host_parts(prep: O.Prepared) -> dict:
+    """The oracle's prepared weight in the canonical host form of a checkpoint
+    (serq_weight_host): row-major E8M0 bytes, residual padded to rp."""
+    r, rp = prep.r, rp_of(prep.r)
+    N, K = prep.qw.shape
+    parts = {"perm": prep.perm.astype(np.int32), "s": prep.s.astype(np.float32),
+             "inv_s": prep.inv_s.astype(np.float32), "wq": O.pack_nibbles(prep.qw)}
+    if prep.fmt == "int4":
+        parts["w_scale"] = prep.sw.astype(np.float32)
+        parts["r_scale"] = prep.sR.astype(np.float32) if r > 0 else np.zeros(N, np.float32)
+        parts["rq"] = O.pack_nibbles(pad_cols(prep.qR, rp)) if r > 0 else np.zeros((N, 0), np.uint8)
+    else:
+        parts["w_scale"] = O.e8m0(prep.Ew)
+        if r > 0:
+            parts["rq"] = O.pack_nibbles(pad_cols(prep.qR, rp))
+            parts["r_scale"] = O.e8m0(pad_cols(prep.ER, rp // 32, fill=-127))
+        else:
+            parts["rq"] = np.zeros((N, 0), np.uint8)
+            parts["r_scale"] = np.zeros((N, 0), np.uint8)
+    return {k: np.ascontiguousarray(v) for k, v in parts.items()}
+
+
+def assert_parts_equal(a: dict, b: dict):
+    for k in ("perm", "s", "inv_s", "wq", "w_scale", "rq", "r_scale"):
+        x, y = np.ascontiguousarray(a[k]), np.ascontiguousarray(b[k])
+        assert x.nbytes == y.nbytes, (k, x.shape, y.shape)
+        assert np.array_equal(x.view(np.uint8).reshape(-1), y.view(np.uint8).reshape(-1)), k

@@ -12,6 +12,7 @@ from .serq import (  # noqa: F401
     alloc_act,
     serq_act_buffer_sizes,
     serq_calib_absmax,
+    serq_debug_fail_next_allocations,
     serq_device_status,
     serq_fold_producer,
     serq_linear,
@@ -20,6 +21,12 @@ from .serq import (  # noqa: F401
     serq_quant_act,
     serq_selftest_wait,
     serq_version,
+    serq_weight_create_from_host,
+    serq_weight_export,
+    serq_weight_file_read,
+    serq_weight_file_write,
     serq_weight_get_view,
+    serq_weight_load,
+    serq_weight_save,
 )
 from ._native import SerqError  # noqa: F401

@@ -32,6 +32,12 @@ class WeightView(ctypes.Structure):
                 ("r_scale", c_void_p), ("r_scale_bytes", c_size_t)]
 
 
+class WeightHost(ctypes.Structure):
+    _fields_ = [("K", c_int), ("N", c_int), ("r", c_int), ("rp", c_int), ("fmt", c_int),
+                ("perm", c_void_p), ("s", c_void_p), ("inv_s", c_void_p), ("wq", c_void_p),
+                ("w_scale", c_void_p), ("rq", c_void_p), ("r_scale", c_void_p)]
+
+
 class ActSizes(ctypes.Structure):
     _fields_ = [("xq", c_size_t), ("xs", c_size_t), ("xsq", c_size_t), ("xss", c_size_t)]
 
@@ -49,6 +55,13 @@ _SIGNATURES = {
                             c_void_p]),
     "serq_linear_small_m_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
+    "serq_weight_export": (c_int, [c_void_p, ctypes.POINTER(WeightHost)]),
+    "serq_weight_create_from_host": (c_int, [ctypes.POINTER(WeightHost), ctypes.POINTER(c_void_p), c_void_p]),
+    "serq_weight_save": (c_int, [c_void_p, c_char_p]),
+    "serq_weight_load": (c_int, [c_char_p, ctypes.POINTER(c_void_p), c_void_p]),
+    "serq_weight_file_write": (c_int, [c_char_p, ctypes.POINTER(WeightHost)]),
+    "serq_weight_file_read": (c_int, [c_char_p, ctypes.POINTER(WeightHost)]),
+    "serq_debug_fail_next_allocations": (c_int, [c_int]),
     "serq_selftest_wait": (c_int, [ctypes.c_longlong, c_int, c_void_p]),
     "serq_device_status": (c_int, [c_void_p]),
     "serq_last_error": (c_char_p, []),

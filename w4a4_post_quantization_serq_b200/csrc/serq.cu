@@ -6,11 +6,13 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <vector>
 
 #include "serq.h"
 
@@ -21,6 +23,7 @@
 #include "gemm_int4.cuh"
 #include "gemm_mxfp4_decode.cuh"
 #include "gemm_mxfp4_pair.cuh"
+#include "weight_format.h"
 
 using namespace serq;
 
@@ -205,7 +208,133 @@ struct serq_weight {
     CUtensorMap tm_r128;
     CUtensorMap tm_wsf;    // wide MXFP4 scales as 256 B rows (box: two 4 KB atom pairs)
     CUtensorMap tm_rsf;
+    float* tmp_b;          // preparation scratch at the end of the arena
+    unsigned int* tmp_col;
 };
+
+namespace {
+
+// Test hook: the next n device allocations of a weight fail with SERQ_ENOMEM
+// without calling cudaMalloc (serq_debug_fail_next_allocations).
+std::atomic<int> g_fail_allocs{0};
+
+serq_status check_weight_shape(int K, int N, int r, int fmt) {
+    if (K < 128 || K % 128 != 0 || K > 32768 || N < 128 || N % 128 != 0 || r < 0 || r > K)
+        return fail(SERQ_EINVAL, "bad shape K=%d N=%d r=%d (need K%%128==0, K<=32768, N%%128==0, 0<=r<=K)", K, N, r);
+    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4) return fail(SERQ_EINVAL, "unknown format %d", fmt);
+    return SERQ_OK;
+}
+
+// One device arena per weight: perm, s, s_perm, inv_s, W^_q and its scales,
+// Q(R) and its scales, the wide MXFP4 scale copies, then preparation scratch.
+// Zero-filled on `cs`. Nothing is left allocated on failure.
+serq_status weight_alloc(int K, int N, int r, int fmt, int dev, cudaStream_t cs, serq_weight** out) {
+    const int rp = residual_width(r);
+    auto* w = new serq_weight();
+    std::memset(w, 0, sizeof(*w));
+    w->K = K;
+    w->N = N;
+    w->r = r;
+    w->rp = rp;
+    w->fmt = fmt;
+    w->device = dev;
+    w->wq_bytes = static_cast<size_t>(N) * (K / 2);
+    w->rq_bytes = static_cast<size_t>(N) * (rp / 2);
+    if (fmt == SERQ_FMT_INT4) {
+        w->wsc_bytes = static_cast<size_t>(N) * 4;
+        w->rsc_bytes = static_cast<size_t>(N) * 4;
+    } else {
+        w->wsc_bytes = atom_bytes(N, K / 32);
+        w->rsc_bytes = rp > 0 ? atom_bytes(N, rp / 32) : 0;
+        const size_t pairs = static_cast<size_t>((N / 128 + 1) / 2);
+        w->wscw_bytes = pairs * (K / 128) * 4096;
+        w->rscw_bytes = rp > 0 ? pairs * ((rp + 127) / 128) * 4096 : 0;
+    }
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        const size_t o = off;
+        off += (bytes + 255) & ~size_t(255);
+        return o;
+    };
+    const size_t o_perm = take(4u * K), o_s = take(4u * K), o_sp = take(4u * K), o_inv = take(4u * K);
+    const size_t o_wq = take(w->wq_bytes), o_wsc = take(w->wsc_bytes);
+    const size_t o_rq = take(w->rq_bytes), o_rsc = take(w->rsc_bytes);
+    const size_t o_wscw = take(w->wscw_bytes), o_rscw = take(w->rscw_bytes);
+    const size_t o_b = take(4u * K), o_col = take(4u * N);
+    int pending = g_fail_allocs.load();
+    while (pending > 0 && !g_fail_allocs.compare_exchange_weak(pending, pending - 1)) {
+    }
+    if (pending > 0) {
+        delete w;
+        return fail(SERQ_ENOMEM, "device allocation of %zu bytes failed (injected by the test hook)", off);
+    }
+    void* arena = nullptr;
+    const cudaError_t ae = cudaMalloc(&arena, off);
+    if (ae != cudaSuccess) {
+        delete w;
+        cudaGetLastError();
+        return fail(SERQ_ENOMEM, "cudaMalloc(%zu) failed: %s", off, cudaGetErrorString(ae));
+    }
+    uint8_t* base = static_cast<uint8_t*>(arena);
+    w->arena = arena;
+    w->perm = reinterpret_cast<int32_t*>(base + o_perm);
+    w->s = reinterpret_cast<float*>(base + o_s);
+    w->s_perm = reinterpret_cast<float*>(base + o_sp);
+    w->inv_s = reinterpret_cast<float*>(base + o_inv);
+    w->wq = base + o_wq;
+    w->wsc = base + o_wsc;
+    w->rq = base + o_rq;
+    w->rsc = base + o_rsc;
+    w->wscw = base + o_wscw;
+    w->rscw = base + o_rscw;
+    w->tmp_b = reinterpret_cast<float*>(base + o_b);
+    w->tmp_col = reinterpret_cast<unsigned int*>(base + o_col);
+    const cudaError_t me = cudaMemsetAsync(arena, 0, off, cs);
+    if (me != cudaSuccess) {
+        cudaFree(arena);
+        delete w;
+        return cuda_fail(me, "cudaMemsetAsync(weight arena)");
+    }
+    *out = w;
+    return SERQ_OK;
+}
+
+// After the packed tensors are in place: the wide MXFP4 scale copies of the
+// CTA-pair kernel, then the tensor maps. Synchronizes `cs`.
+serq_status weight_finish(serq_weight* w, cudaStream_t cs) {
+    const int K = w->K, N = w->N, rp = w->rp, fmt = w->fmt;
+    if (fmt == SERQ_FMT_MXFP4) {
+        scale_widen_kernel<<<static_cast<unsigned>((w->wscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
+            static_cast<const uint8_t*>(w->wsc), N / 128, K / 128, w->wscw, w->wscw_bytes);
+        if (rp > 0)
+            scale_widen_kernel<<<static_cast<unsigned>((w->rscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
+                static_cast<const uint8_t*>(w->rsc), N / 128, (rp + 127) / 128, w->rscw, w->rscw_bytes);
+        SERQ_CUDA(cudaGetLastError());
+    }
+    SERQ_CUDA(cudaStreamSynchronize(cs));
+    const uint32_t bi = box_inner_bytes(fmt);
+    const bool swz = fmt == SERQ_FMT_MXFP4;
+    if (serq_status st = make_map(&w->tm_w, w->wq, K / 2, N, bi, 256, swz)) return st;
+    if (rp > 0) {
+        if (serq_status st = make_map(&w->tm_r, w->rq, rp / 2, N, bi, 256, swz)) return st;
+    } else {
+        w->tm_r = w->tm_w;
+    }
+    if (fmt == SERQ_FMT_MXFP4) {
+        if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return st;
+        if (serq_status st = make_map(&w->tm_wsf, w->wscw, 256, w->wscw_bytes / 256, 256, 32, false)) return st;
+        if (rp > 0) {
+            if (serq_status st = make_map(&w->tm_rsf, w->rscw, 256, w->rscw_bytes / 256, 256, 32, false)) return st;
+            if (serq_status st = make_map(&w->tm_r128, w->rq, rp / 2, N, 128, 128, true)) return st;
+        } else {
+            w->tm_rsf = w->tm_wsf;
+            w->tm_r128 = w->tm_w128;
+        }
+    }
+    return SERQ_OK;
+}
+
+}  // namespace
 
 // ============================================================== allocation-free small-M entry
 // Scratch of serq_linear_small_m_noalloc: split-K tickets (first 4 KiB, one
@@ -305,10 +434,7 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     if (desc == nullptr || out == nullptr) return fail(SERQ_EINVAL, "NULL argument");
     *out = nullptr;
     const int K = desc->K, N = desc->N, r = desc->r, fmt = desc->fmt;
-    if (K < 128 || K % 128 != 0 || K > 32768 || N < 128 || N % 128 != 0 || r < 0 || r > K)
-        return fail(SERQ_EINVAL, "bad shape K=%d N=%d r=%d (need K%%128==0, K<=32768, N%%128==0, 0<=r<=K)", K, N,
-                    r);
-    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4) return fail(SERQ_EINVAL, "unknown format %d", fmt);
+    if (serq_status st = check_weight_shape(K, N, r, fmt)) return st;
     if (desc->W == nullptr || !aligned16(desc->W)) return fail(SERQ_EINVAL, "W must be a 16-byte aligned pointer");
     if ((desc->act_absmax == nullptr) == (desc->s == nullptr))
         return fail(SERQ_EINVAL, "give exactly one of act_absmax and s");
@@ -317,62 +443,11 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     if (serq_status st = device_check(&dev, &info)) return st;
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
-    const int rp = residual_width(r);
-    auto* w = new serq_weight();
-    std::memset(w, 0, sizeof(*w));
-    w->K = K;
-    w->N = N;
-    w->r = r;
-    w->rp = rp;
-    w->fmt = fmt;
-    w->device = dev;
-    w->wq_bytes = static_cast<size_t>(N) * (K / 2);
-    w->rq_bytes = static_cast<size_t>(N) * (rp / 2);
-    if (fmt == SERQ_FMT_INT4) {
-        w->wsc_bytes = static_cast<size_t>(N) * 4;
-        w->rsc_bytes = static_cast<size_t>(N) * 4;
-    } else {
-        w->wsc_bytes = atom_bytes(N, K / 32);
-        w->rsc_bytes = rp > 0 ? atom_bytes(N, rp / 32) : 0;
-        const size_t pairs = static_cast<size_t>((N / 128 + 1) / 2);
-        w->wscw_bytes = pairs * (K / 128) * 4096;
-        w->rscw_bytes = rp > 0 ? pairs * ((rp + 127) / 128) * 4096 : 0;
-    }
-    // one arena: perm, s, s_perm, inv_s, wq, wsc, rq, rsc, then scratch
-    size_t off = 0;
-    auto take = [&](size_t bytes) {
-        const size_t o = off;
-        off += (bytes + 255) & ~size_t(255);
-        return o;
-    };
-    const size_t o_perm = take(4u * K), o_s = take(4u * K), o_sp = take(4u * K), o_inv = take(4u * K);
-    const size_t o_wq = take(w->wq_bytes), o_wsc = take(w->wsc_bytes);
-    const size_t o_rq = take(w->rq_bytes), o_rsc = take(w->rsc_bytes);
-    const size_t o_wscw = take(w->wscw_bytes), o_rscw = take(w->rscw_bytes);
-    const size_t keep = off;
-    const size_t o_b = take(4u * K), o_col = take(4u * N);
-    void* arena = nullptr;
-    const cudaError_t ae = cudaMalloc(&arena, off);
-    if (ae != cudaSuccess) {
-        delete w;
-        cudaGetLastError();
-        return fail(SERQ_ENOMEM, "cudaMalloc(%zu) failed: %s", off, cudaGetErrorString(ae));
-    }
-    (void)keep;
-    uint8_t* base = static_cast<uint8_t*>(arena);
-    w->arena = arena;
-    w->perm = reinterpret_cast<int32_t*>(base + o_perm);
-    w->s = reinterpret_cast<float*>(base + o_s);
-    w->s_perm = reinterpret_cast<float*>(base + o_sp);
-    w->inv_s = reinterpret_cast<float*>(base + o_inv);
-    w->wq = base + o_wq;
-    w->wsc = base + o_wsc;
-    w->rq = base + o_rq;
-    w->rsc = base + o_rsc;
-    w->wscw = base + o_wscw;
-    w->rscw = base + o_rscw;
-    float* tmp_b = reinterpret_cast<float*>(base + o_b);
-    unsigned int* tmp_col = reinterpret_cast<unsigned int*>(base + o_col);
+    serq_weight* w = nullptr;
+    if (serq_status st = weight_alloc(K, N, r, fmt, dev, cs, &w)) return st;
+    const int rp = w->rp;
+    float* tmp_b = w->tmp_b;
+    unsigned int* tmp_col = w->tmp_col;
 
     auto bail = [&](serq_status st) {
         cudaStreamSynchronize(cs);
@@ -386,7 +461,6 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     } while (0)
 
     const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(desc->W);
-    PREP_CUDA(cudaMemsetAsync(arena, 0, off, cs));
     // Stage 1: SAF scales
     if (desc->act_absmax != nullptr) {
         row_absmax_kernel<<<(K + 7) / 8, 256, 0, cs>>>(W, K, N, tmp_b);
@@ -416,38 +490,9 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
         if (r > 0)
             residual_mxfp4_kernel<<<dim3(N / 32, (rp / 32 + 7) / 8), qblock, 0, cs>>>(
                 W, w->perm, w->s_perm, K, N, r, rp, w->rq, static_cast<uint8_t*>(w->rsc));
-        scale_widen_kernel<<<static_cast<unsigned>((w->wscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
-            static_cast<const uint8_t*>(w->wsc), N / 128, K / 128, w->wscw, w->wscw_bytes);
-        if (rp > 0)
-            scale_widen_kernel<<<static_cast<unsigned>((w->rscw_bytes / 16 + 255) / 256), 256, 0, cs>>>(
-                static_cast<const uint8_t*>(w->rsc), N / 128, (rp + 127) / 128, w->rscw, w->rscw_bytes);
     }
     PREP_CUDA(cudaGetLastError());
-    PREP_CUDA(cudaStreamSynchronize(cs));
-
-    const uint32_t bi = box_inner_bytes(fmt);
-    const bool swz = fmt == SERQ_FMT_MXFP4;
-    if (serq_status st = make_map(&w->tm_w, w->wq, K / 2, N, bi, 256, swz)) return bail(st);
-    if (rp > 0) {
-        if (serq_status st = make_map(&w->tm_r, w->rq, rp / 2, N, bi, 256, swz)) return bail(st);
-    } else {
-        w->tm_r = w->tm_w;
-    }
-    if (fmt == SERQ_FMT_MXFP4) {
-        if (serq_status st = make_map(&w->tm_w128, w->wq, K / 2, N, 128, 128, true)) return bail(st);
-        if (serq_status st = make_map(&w->tm_wsf, w->wscw, 256, w->wscw_bytes / 256, 256, 32, false)) return bail(st);
-        if (rp > 0) {
-            if (serq_status st = make_map(&w->tm_rsf, w->rscw, 256, w->rscw_bytes / 256, 256, 32, false))
-                return bail(st);
-        } else {
-            w->tm_rsf = w->tm_wsf;
-        }
-        if (rp > 0) {
-            if (serq_status st = make_map(&w->tm_r128, w->rq, rp / 2, N, 128, 128, true)) return bail(st);
-        } else {
-            w->tm_r128 = w->tm_w128;
-        }
-    }
+    if (serq_status st = weight_finish(w, cs)) return bail(st);
 #undef PREP_CUDA
     *out = w;
     return SERQ_OK;
@@ -473,6 +518,336 @@ serq_status serq_weight_get_view(const serq_weight* w, serq_weight_view* out) {
     out->r_scale_bytes = w->rsc_bytes;
     return SERQ_OK;
 }
+
+}  // extern "C"
+
+// ============================================================== checkpoint / export / import
+namespace {
+
+bool is_int4_code_ok(uint8_t nib) { return (nib & 0xF) != 0x8; }  // -8 never occurs
+
+// Checks the canonical host form (see serq_weight_host in serq.h).
+serq_status check_host_weight(const serq_weight_host* h) {
+    if (serq_status st = check_weight_shape(h->K, h->N, h->r, h->fmt)) return st;
+    const int K = h->K, N = h->N, r = h->r, rp = h->rp, fmt = h->fmt;
+    if (rp != residual_width(r)) return fail(SERQ_EINVAL, "rp=%d, expected round_up(r, 64) = %d", rp, residual_width(r));
+    if (h->perm == nullptr || h->s == nullptr || h->inv_s == nullptr || h->wq == nullptr || h->w_scale == nullptr)
+        return fail(SERQ_EINVAL, "NULL part (perm, s, inv_s, wq and w_scale are required)");
+    if (rp > 0 && (h->rq == nullptr || h->r_scale == nullptr)) return fail(SERQ_EINVAL, "r > 0 needs rq and r_scale");
+    std::vector<uint8_t> seen(static_cast<size_t>(K), 0);
+    for (int i = 0; i < K; ++i) {
+        const int j = h->perm[i];
+        if (j < 0 || j >= K || seen[j]) return fail(SERQ_EINVAL, "perm is not a permutation of 0..K-1 (at %d)", i);
+        seen[j] = 1;
+    }
+    for (int j = 0; j < K; ++j)
+        if (!std::isfinite(h->s[j]) || !(h->s[j] > 0.0f)) return fail(SERQ_EINVAL, "s[%d] is not finite and > 0", j);
+    for (int i = 0; i < K; ++i) {
+        const float want = 1.0f / h->s[h->perm[i]];
+        if (std::memcmp(&want, &h->inv_s[i], 4) != 0) return fail(SERQ_EINVAL, "inv_s[%d] != 1/s[perm[%d]]", i, i);
+    }
+    const size_t wq_bytes = static_cast<size_t>(N) * (K / 2);
+    const size_t rq_row = static_cast<size_t>(rp / 2);
+    if (fmt == SERQ_FMT_INT4) {
+        for (size_t i = 0; i < wq_bytes; ++i)
+            if (!is_int4_code_ok(h->wq[i]) || !is_int4_code_ok(h->wq[i] >> 4))
+                return fail(SERQ_EINVAL, "INT4 code -8 in wq (byte %zu)", i);
+        const float* ws = static_cast<const float*>(h->w_scale);
+        for (int n = 0; n < N; ++n)
+            if (!std::isfinite(ws[n]) || ws[n] < 0.0f) return fail(SERQ_EINVAL, "w_scale[%d] not finite >= 0", n);
+        if (h->r_scale != nullptr) {
+            const float* rs = static_cast<const float*>(h->r_scale);
+            for (int n = 0; n < N; ++n)
+                if (!std::isfinite(rs[n]) || rs[n] < 0.0f || (rp == 0 && rs[n] != 0.0f))
+                    return fail(SERQ_EINVAL, "r_scale[%d] not finite >= 0 (or nonzero with r = 0)", n);
+        }
+    } else {
+        const uint8_t* ws = static_cast<const uint8_t*>(h->w_scale);
+        for (size_t i = 0; i < static_cast<size_t>(N) * (K / 32); ++i)
+            if (ws[i] == 0xFF) return fail(SERQ_EINVAL, "E8M0 byte 0xFF in w_scale");
+        if (rp > 0) {
+            const uint8_t* rs = static_cast<const uint8_t*>(h->r_scale);
+            const int nbr = rp / 32, used = (r + 31) / 32;
+            for (int n = 0; n < N; ++n)
+                for (int b = 0; b < nbr; ++b) {
+                    const uint8_t e = rs[static_cast<size_t>(n) * nbr + b];
+                    if (e == 0xFF || (b >= used && e != 0))
+                        return fail(SERQ_EINVAL, "r_scale row %d block %d: 0xFF or nonzero past r", n, b);
+                }
+        }
+    }
+    for (int n = 0; n < N && rp > 0; ++n)
+        for (int c = r; c < rp; ++c) {
+            const uint8_t byte = h->rq[static_cast<size_t>(n) * rq_row + c / 2];
+            const uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
+            if (nib != 0) return fail(SERQ_EINVAL, "rq row %d: nonzero code at position %d >= r", n, c);
+        }
+    if (fmt == SERQ_FMT_INT4 && rp > 0)
+        for (size_t i = 0; i < static_cast<size_t>(N) * rq_row; ++i)
+            if (!is_int4_code_ok(h->rq[i]) || !is_int4_code_ok(h->rq[i] >> 4))
+                return fail(SERQ_EINVAL, "INT4 code -8 in rq (byte %zu)", i);
+    return SERQ_OK;
+}
+
+// Owning host copy of the canonical parts.
+struct HostWeight {
+    serq_weight_host h{};
+    std::vector<uint8_t> buf;
+    void allocate(int fmt, int K, int N, int r, int rp) {
+        const wfmt::Sizes z = wfmt::canonical_sizes(fmt, K, N, rp);
+        buf.assign(z.total(), 0);
+        uint8_t* p = buf.data();
+        h.K = K;
+        h.N = N;
+        h.r = r;
+        h.rp = rp;
+        h.fmt = fmt;
+        h.perm = reinterpret_cast<int32_t*>(p);
+        p += z.perm;
+        h.s = reinterpret_cast<float*>(p);
+        p += z.s;
+        h.inv_s = reinterpret_cast<float*>(p);
+        p += z.inv_s;
+        h.wq = p;
+        p += z.wq;
+        h.w_scale = p;
+        p += z.w_scale;
+        h.rq = z.rq > 0 ? p : nullptr;
+        p += z.rq;
+        h.r_scale = z.r_scale > 0 ? p : nullptr;
+    }
+};
+
+struct FileCloser {
+    FILE* f;
+    ~FileCloser() {
+        if (f != nullptr) fclose(f);
+    }
+};
+
+serq_status write_file(const char* path, const serq_weight_host* h) {
+    const wfmt::Sizes z = wfmt::canonical_sizes(h->fmt, h->K, h->N, h->rp);
+    const void* parts[7] = {h->perm, h->s, h->inv_s, h->wq, h->w_scale, h->rq, h->r_scale};
+    const size_t sizes[7] = {z.perm, z.s, z.inv_s, z.wq, z.w_scale, z.rq, z.r_scale};
+    std::vector<uint8_t> zeros;
+    wfmt::Header hd;
+    std::memset(&hd, 0, sizeof(hd));
+    std::memcpy(hd.magic, wfmt::kMagic, 8);
+    hd.version = wfmt::kVersion;
+    hd.fmt = h->fmt;
+    hd.K = h->K;
+    hd.N = h->N;
+    hd.r = h->r;
+    hd.rp = h->rp;
+    hd.payload_bytes = z.total();
+    uint64_t ck = 1469598103934665603ull;
+    for (int i = 0; i < 7; ++i) {
+        if (sizes[i] == 0) continue;
+        const uint8_t* src = static_cast<const uint8_t*>(parts[i]);
+        if (src == nullptr) {  // only r_scale of INT4 with r = 0 may be absent: zeros
+            zeros.assign(sizes[i], 0);
+            src = zeros.data();
+        }
+        ck = wfmt::fnv1a64(src, sizes[i], ck);
+    }
+    hd.checksum = ck;
+    FileCloser fc{fopen(path, "wb")};
+    if (fc.f == nullptr) return fail(SERQ_EINVAL, "cannot open %s for writing", path);
+    if (fwrite(&hd, sizeof(hd), 1, fc.f) != 1) return fail(SERQ_EINVAL, "write to %s failed", path);
+    for (int i = 0; i < 7; ++i) {
+        if (sizes[i] == 0) continue;
+        const void* src = parts[i];
+        if (src == nullptr) {
+            zeros.assign(sizes[i], 0);
+            src = zeros.data();
+        }
+        if (fwrite(src, 1, sizes[i], fc.f) != sizes[i]) return fail(SERQ_EINVAL, "write to %s failed", path);
+    }
+    if (fclose(fc.f) != 0) {
+        fc.f = nullptr;
+        return fail(SERQ_EINVAL, "closing %s failed", path);
+    }
+    fc.f = nullptr;
+    return SERQ_OK;
+}
+
+// Reads and checks a checkpoint into an owning host copy.
+serq_status read_file(const char* path, HostWeight* hw) {
+    FileCloser fc{fopen(path, "rb")};
+    if (fc.f == nullptr) return fail(SERQ_EINVAL, "cannot open %s", path);
+    wfmt::Header hd;
+    if (fread(&hd, sizeof(hd), 1, fc.f) != 1) return fail(SERQ_EINVAL, "%s: truncated header", path);
+    if (std::memcmp(hd.magic, wfmt::kMagic, 8) != 0) return fail(SERQ_EINVAL, "%s: not a SERQ weight file", path);
+    if (hd.version != wfmt::kVersion) return fail(SERQ_EINVAL, "%s: unsupported version %u", path, hd.version);
+    if (serq_status st = check_weight_shape(hd.K, hd.N, hd.r, hd.fmt)) return st;
+    if (hd.rp != residual_width(hd.r)) return fail(SERQ_EINVAL, "%s: inconsistent rp", path);
+    const wfmt::Sizes z = wfmt::canonical_sizes(hd.fmt, hd.K, hd.N, hd.rp);
+    if (hd.payload_bytes != z.total()) return fail(SERQ_EINVAL, "%s: payload size mismatch", path);
+    hw->allocate(hd.fmt, hd.K, hd.N, hd.r, hd.rp);
+    if (fread(hw->buf.data(), 1, hw->buf.size(), fc.f) != hw->buf.size())
+        return fail(SERQ_EINVAL, "%s: truncated payload", path);
+    if (fgetc(fc.f) != EOF) return fail(SERQ_EINVAL, "%s: trailing bytes after the payload", path);
+    if (wfmt::fnv1a64(hw->buf.data(), hw->buf.size()) != hd.checksum) return fail(SERQ_EINVAL, "%s: checksum mismatch", path);
+    return check_host_weight(&hw->h);
+}
+
+serq_status copy_parts(const serq_weight_host* src, serq_weight_host* dst) {
+    const wfmt::Sizes z = wfmt::canonical_sizes(src->fmt, src->K, src->N, src->rp);
+    dst->K = src->K;
+    dst->N = src->N;
+    dst->r = src->r;
+    dst->rp = src->rp;
+    dst->fmt = src->fmt;
+    auto cp = [](void* d, const void* s, size_t n) {
+        if (d != nullptr && n > 0) {
+            if (s != nullptr)
+                std::memcpy(d, s, n);
+            else
+                std::memset(d, 0, n);
+        }
+    };
+    cp(dst->perm, src->perm, z.perm);
+    cp(dst->s, src->s, z.s);
+    cp(dst->inv_s, src->inv_s, z.inv_s);
+    cp(dst->wq, src->wq, z.wq);
+    cp(dst->w_scale, src->w_scale, z.w_scale);
+    cp(dst->rq, src->rq, z.rq);
+    cp(dst->r_scale, src->r_scale, z.r_scale);
+    return SERQ_OK;
+}
+
+// Runs `fn` with the weight's device current, restoring the caller's device.
+template <class F>
+serq_status on_device(int dev, F&& fn) {
+    int cur = -1;
+    SERQ_CUDA(cudaGetDevice(&cur));
+    if (cur != dev) SERQ_CUDA(cudaSetDevice(dev));
+    const serq_status st = fn();
+    if (cur != dev) cudaSetDevice(cur);
+    return st;
+}
+
+}  // namespace
+
+extern "C" {
+
+serq_status serq_weight_export(const serq_weight* w, serq_weight_host* dst) {
+    if (w == nullptr || dst == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    dst->K = w->K;
+    dst->N = w->N;
+    dst->r = w->r;
+    dst->rp = w->rp;
+    dst->fmt = w->fmt;
+    return on_device(w->device, [&]() -> serq_status {
+        SERQ_CUDA(cudaDeviceSynchronize());
+        const int K = w->K, N = w->N, rp = w->rp;
+        if (dst->perm != nullptr) SERQ_CUDA(cudaMemcpy(dst->perm, w->perm, 4u * K, cudaMemcpyDeviceToHost));
+        if (dst->s != nullptr) SERQ_CUDA(cudaMemcpy(dst->s, w->s, 4u * K, cudaMemcpyDeviceToHost));
+        if (dst->inv_s != nullptr) SERQ_CUDA(cudaMemcpy(dst->inv_s, w->inv_s, 4u * K, cudaMemcpyDeviceToHost));
+        if (dst->wq != nullptr) SERQ_CUDA(cudaMemcpy(dst->wq, w->wq, w->wq_bytes, cudaMemcpyDeviceToHost));
+        if (dst->rq != nullptr && w->rq_bytes > 0)
+            SERQ_CUDA(cudaMemcpy(dst->rq, w->rq, w->rq_bytes, cudaMemcpyDeviceToHost));
+        if (w->fmt == SERQ_FMT_INT4) {
+            if (dst->w_scale != nullptr) SERQ_CUDA(cudaMemcpy(dst->w_scale, w->wsc, 4u * N, cudaMemcpyDeviceToHost));
+            if (dst->r_scale != nullptr) SERQ_CUDA(cudaMemcpy(dst->r_scale, w->rsc, 4u * N, cudaMemcpyDeviceToHost));
+        } else {
+            std::vector<uint8_t> atoms;
+            if (dst->w_scale != nullptr) {
+                atoms.resize(w->wsc_bytes);
+                SERQ_CUDA(cudaMemcpy(atoms.data(), w->wsc, w->wsc_bytes, cudaMemcpyDeviceToHost));
+                wfmt::atoms_to_rows(atoms.data(), N, K / 32, static_cast<uint8_t*>(dst->w_scale));
+            }
+            if (dst->r_scale != nullptr && rp > 0) {
+                atoms.resize(w->rsc_bytes);
+                SERQ_CUDA(cudaMemcpy(atoms.data(), w->rsc, w->rsc_bytes, cudaMemcpyDeviceToHost));
+                wfmt::atoms_to_rows(atoms.data(), N, rp / 32, static_cast<uint8_t*>(dst->r_scale));
+            }
+        }
+        return SERQ_OK;
+    });
+}
+
+serq_status serq_weight_create_from_host(const serq_weight_host* src, serq_weight** out, serq_stream stream) {
+    if (src == nullptr || out == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    *out = nullptr;
+    if (serq_status st = check_host_weight(src)) return st;
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int K = src->K, N = src->N, rp = src->rp;
+    serq_weight* w = nullptr;
+    if (serq_status st = weight_alloc(K, N, src->r, src->fmt, dev, cs, &w)) return st;
+    auto bail = [&](serq_status st) {
+        cudaStreamSynchronize(cs);
+        serq_weight_destroy(w);
+        return st;
+    };
+    std::vector<float> s_perm(static_cast<size_t>(K));
+    for (int i = 0; i < K; ++i) s_perm[i] = src->s[src->perm[i]];
+    std::vector<uint8_t> watoms, ratoms;
+    auto up = [&](void* d, const void* h, size_t n) -> serq_status {
+        if (n == 0) return SERQ_OK;
+        const cudaError_t e = cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, cs);
+        return e == cudaSuccess ? SERQ_OK : cuda_fail(e, "cudaMemcpyAsync(weight upload)");
+    };
+    serq_status st = up(w->perm, src->perm, 4u * K);
+    if (!st) st = up(w->s, src->s, 4u * K);
+    if (!st) st = up(w->s_perm, s_perm.data(), 4u * K);
+    if (!st) st = up(w->inv_s, src->inv_s, 4u * K);
+    if (!st) st = up(w->wq, src->wq, w->wq_bytes);
+    if (!st && rp > 0) st = up(w->rq, src->rq, w->rq_bytes);
+    if (!st) {
+        if (src->fmt == SERQ_FMT_INT4) {
+            st = up(w->wsc, src->w_scale, 4u * N);
+            if (!st && src->r_scale != nullptr) st = up(w->rsc, src->r_scale, 4u * N);
+        } else {
+            watoms.resize(w->wsc_bytes);
+            wfmt::rows_to_atoms(static_cast<const uint8_t*>(src->w_scale), N, K / 32, watoms.data());
+            st = up(w->wsc, watoms.data(), w->wsc_bytes);
+            if (!st && rp > 0) {
+                ratoms.resize(w->rsc_bytes);
+                wfmt::rows_to_atoms(static_cast<const uint8_t*>(src->r_scale), N, rp / 32, ratoms.data());
+                st = up(w->rsc, ratoms.data(), w->rsc_bytes);
+            }
+        }
+    }
+    if (!st) st = weight_finish(w, cs);  // synchronizes: the pageable host copies are complete
+    if (st) return bail(st);
+    *out = w;
+    return SERQ_OK;
+}
+
+serq_status serq_weight_save(const serq_weight* w, const char* path) {
+    if (w == nullptr || path == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    HostWeight hw;
+    hw.allocate(w->fmt, w->K, w->N, w->r, w->rp);
+    if (serq_status st = serq_weight_export(w, &hw.h)) return st;
+    return write_file(path, &hw.h);
+}
+
+serq_status serq_weight_load(const char* path, serq_weight** out, serq_stream stream) {
+    if (path == nullptr || out == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    *out = nullptr;
+    HostWeight hw;
+    if (serq_status st = read_file(path, &hw)) return st;
+    return serq_weight_create_from_host(&hw.h, out, stream);
+}
+
+serq_status serq_weight_file_write(const char* path, const serq_weight_host* src) {
+    if (path == nullptr || src == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    if (serq_status st = check_host_weight(src)) return st;
+    return write_file(path, src);
+}
+
+serq_status serq_weight_file_read(const char* path, serq_weight_host* dst) {
+    if (path == nullptr || dst == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    HostWeight hw;
+    if (serq_status st = read_file(path, &hw)) return st;
+    return copy_parts(&hw.h, dst);
+}
+
+int serq_debug_fail_next_allocations(int n) { return g_fail_allocs.exchange(n < 0 ? 0 : n); }
 
 serq_status serq_fold_producer(const serq_weight* w, const void* src, int rows, void* dst, serq_stream stream) {
     if (w == nullptr || src == nullptr || dst == nullptr) return fail(SERQ_EINVAL, "NULL argument");

@@ -9,9 +9,11 @@ no sm_100 device is present.
 from __future__ import annotations
 
 import ctypes
+import os
 from dataclasses import dataclass
 from typing import Dict, Optional
 
+import numpy as np
 import torch
 
 from . import _native as N
@@ -106,6 +108,88 @@ def serq_weight_get_view(w: SerqWeight) -> Dict[str, torch.Tensor]:
             out["rq"] = _view(v.rq, (v.N, v.rp // 2), "|u1", w)
             out["r_scale"] = _view(v.r_scale, (v.r_scale_bytes,), "|u1", w)
     return out
+
+
+def _host_parts(K: int, N_: int, r: int, rp: int, fmt: int) -> Dict[str, np.ndarray]:
+    """Zeroed numpy buffers of the canonical host form (see serq_weight_host in serq.h)."""
+    out = {"perm": np.zeros(K, np.int32), "s": np.zeros(K, np.float32), "inv_s": np.zeros(K, np.float32),
+           "wq": np.zeros((N_, K // 2), np.uint8), "rq": np.zeros((N_, rp // 2), np.uint8)}
+    if fmt == 0:
+        out["w_scale"] = np.zeros(N_, np.float32)
+        out["r_scale"] = np.zeros(N_, np.float32)
+    else:
+        out["w_scale"] = np.zeros((N_, K // 32), np.uint8)
+        out["r_scale"] = np.zeros((N_, rp // 32), np.uint8)
+    return out
+
+
+def _host_struct(parts: Dict[str, np.ndarray], K: int, N_: int, r: int, rp: int, fmt: int):
+    """serq_weight_host pointing into contiguous numpy arrays (kept alive by the caller)."""
+    def p(name):
+        a = parts.get(name)
+        if a is None or a.size == 0:
+            return None
+        if not a.flags["C_CONTIGUOUS"]:
+            raise ValueError(f"{name} must be C-contiguous")
+        return a.ctypes.data
+    return N.WeightHost(K, N_, r, rp, fmt, p("perm"), p("s"), p("inv_s"), p("wq"), p("w_scale"), p("rq"),
+                        p("r_scale"))
+
+
+def serq_weight_export(w: SerqWeight) -> Dict[str, np.ndarray]:
+    """Canonical host copies of a prepared weight (perm, s, inv_s, wq, w_scale, rq, r_scale)."""
+    parts = _host_parts(w.K, w.N, w.r, w.rp, w.fmt)
+    st = _host_struct(parts, w.K, w.N, w.r, w.rp, w.fmt)
+    N.check(N.load().serq_weight_export(w.handle, ctypes.byref(st)))
+    return parts
+
+
+def serq_weight_create_from_host(parts: Dict[str, np.ndarray], K: int, N_: int, r: int, fmt,
+                                 stream=None) -> SerqWeight:
+    """A prepared weight on the current device from canonical host arrays. Synchronizes."""
+    f = _fmt(fmt)
+    rp = ((r + 63) // 64) * 64 if r > 0 else 0
+    keep = {k: np.ascontiguousarray(v) for k, v in parts.items() if v is not None}
+    st = _host_struct(keep, K, N_, r, rp, f)
+    h = ctypes.c_void_p()
+    N.check(N.load().serq_weight_create_from_host(ctypes.byref(st), ctypes.byref(h), _stream(stream)))
+    return SerqWeight(h.value, K, N_, r, f)
+
+
+def serq_weight_save(w: SerqWeight, path: str) -> None:
+    N.check(N.load().serq_weight_save(w.handle, os.fsencode(path)))
+
+
+def serq_weight_load(path: str, stream=None) -> SerqWeight:
+    h = ctypes.c_void_p()
+    N.check(N.load().serq_weight_load(os.fsencode(path), ctypes.byref(h), _stream(stream)))
+    info = N.WeightHost()
+    N.check(N.load().serq_weight_export(h, ctypes.byref(info)))
+    return SerqWeight(h.value, info.K, info.N, info.r, info.fmt)
+
+
+def serq_weight_file_write(path: str, parts: Dict[str, np.ndarray], K: int, N_: int, r: int, fmt) -> None:
+    """Write a checkpoint from canonical host arrays (no GPU needed)."""
+    f = _fmt(fmt)
+    rp = ((r + 63) // 64) * 64 if r > 0 else 0
+    keep = {k: np.ascontiguousarray(v) for k, v in parts.items() if v is not None}
+    st = _host_struct(keep, K, N_, r, rp, f)
+    N.check(N.load().serq_weight_file_write(os.fsencode(path), ctypes.byref(st)))
+
+
+def serq_weight_file_read(path: str):
+    """Read a checkpoint into canonical host arrays (no GPU needed): (parts, K, N, r, fmt)."""
+    info = N.WeightHost()
+    N.check(N.load().serq_weight_file_read(os.fsencode(path), ctypes.byref(info)))
+    parts = _host_parts(info.K, info.N, info.r, info.rp, info.fmt)
+    st = _host_struct(parts, info.K, info.N, info.r, info.rp, info.fmt)
+    N.check(N.load().serq_weight_file_read(os.fsencode(path), ctypes.byref(st)))
+    return parts, info.K, info.N, info.r, info.fmt
+
+
+def serq_debug_fail_next_allocations(n: int) -> int:
+    """Test hook: the next n weight allocations fail with SERQ_ENOMEM (no cudaMalloc)."""
+    return int(N.load().serq_debug_fail_next_allocations(int(n)))
 
 
 def serq_fold_producer(w: SerqWeight, src: torch.Tensor, dst: Optional[torch.Tensor] = None,
