@@ -45,6 +45,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-clocks", action="store_true", help="do not sample nvidia-smi (for profiler runs)")
     ap.add_argument("--only", default=None, help="time only the named linear of the workload (profiling)")
+    ap.add_argument("--workload", default=WORKLOAD, choices=[WORKLOAD, "qproj_int4"],
+                    help="the step's workload (default: the MXFP4 MLP); qproj_int4 is for profiling the INT4 kernel")
     ap.add_argument("--profile-decode", default=None, metavar="SHAPE",
                     help="run a few plain small-M launches of one decode shape (q, kv, gate_up, down) at "
                          "--decode-m tokens and exit (for profilers)")
@@ -100,7 +102,7 @@ def max_over_ranks(pg, value: float) -> float:
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """NVML samples (every 10 ms) of the SM clock, power and clock-event reasons.
+    """NVML samples (every `period_s`, 1 ms by default) of the SM clock, power and clock-event reasons.
 
     Read-only queries; sampling runs in a thread from start() to stop().
     """
@@ -111,8 +113,9 @@ class ClockSampler:
                ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
                ("hw_power_brake", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
 
-    def __init__(self, device_index: int):
+    def __init__(self, device_index: int, period_s: float = 0.001):
         import threading
+        self.period = period_s
         self.samples = []
         self.window = None
         self._stop = threading.Event()
@@ -138,7 +141,7 @@ class ClockSampler:
                                      nv.nvmlDeviceGetPowerUsage(self.h) / 1000.0))
             except Exception:
                 pass
-            time.sleep(0.01)
+            time.sleep(self.period)
 
     def mark(self, t0, t1):
         self.window = (t0, t1)
@@ -161,7 +164,8 @@ class ClockSampler:
                 "power_w_max": max(s[3] for s in self.samples), "samples": len(self.samples),
                 "samples_in_timed_region": len(inside),
                 "sm_mhz_timed_region": statistics.median(s[1] for s in inside) if inside else None,
-                "reasons": sorted(reasons), "source": "NVML, 10 ms period, 0.5 s pre-roll + timed region"}
+                "reasons": sorted(reasons),
+                "source": f"NVML, {self.period * 1e3:g} ms period, 0.5 s pre-roll + timed region"}
 
 
 # ----------------------------------------------------------------- workload
@@ -189,19 +193,50 @@ def build_layers(wl, r_override=None, device="cuda"):
     return layers
 
 
-def run_step(layers, gemm_events=None):
+def quant_act_bytes(M: int, K: int, r: int, fmt: str) -> int:
+    """Algorithmic HBM bytes of one serq_quant_act: read X^ (bf16), write the
+    packed codes of X^_q and X~_{s,q} and their scales."""
+    rp = ((r + 63) // 64) * 64 if r > 0 else 0
+    scales = (M * K // 32 + M * rp // 32) if fmt == "mxfp4" else (4 * M + (4 * M if rp else 0))
+    return 2 * M * K + M * K // 2 + M * rp // 2 + scales
+
+
+def quant_roofline(layers, quant_ms, hbm_gbs):
+    """HBM roofline of serq_quant_act over the step's launches (CUDA events)."""
+    if not quant_ms:
+        return None
+    nbytes = [quant_act_bytes(L["qa"].M, L["lin"].K, L["r"], L["lin"].fmt) for L in layers]
+    tot_b, tot_ms = sum(nbytes), sum(quant_ms)
+    return {"bound": "hbm", "kernel": "quant_act", "bytes_per_step": tot_b,
+            "us_per_step": round(tot_ms * 1e3, 2), "achieved": tot_b / (tot_ms * 1e-3) / 1e9, "unit": "GB/s",
+            "peak": hbm_gbs, "frac": tot_b / (tot_ms * 1e-3) / 1e9 / hbm_gbs,
+            "per_launch": {L["lin"].name: {"bytes": b, "us": round(t * 1e3, 2),
+                                           "GBs": round(b / (t * 1e-3) / 1e9, 1)}
+                           for L, b, t in zip(layers, nbytes, quant_ms)}}
+
+
+def run_step(layers, events=None):
+    """One step: per linear, serq_quant_act then serq_linear. With `events`
+    ([layer][3] CUDA events) the quant launch is bracketed by events 0-1 and
+    the linear by events 1-2, on the launching (current) stream."""
     import w4a4_post_quantization_serq_b200 as S
     for i, L in enumerate(layers):
+        if events is not None:
+            events[i][0].record()
         S.serq_quant_act(L["Xh"], L["r"], L["lin"].fmt, out=L["qa"])
-        if gemm_events is not None:
-            gemm_events[i][0].record()
+        if events is not None:
+            events[i][1].record()
         S.serq_linear(L["w"], L["qa"], Y=L["Y"])
-        if gemm_events is not None:
-            gemm_events[i][1].record()
+        if events is not None:
+            events[i][2].record()
 
 
 def time_steps(layers, steps, warmup, pg, per_gemm=True, sampler=None):
-    """Device time of `steps` steps (CUDA events on the launching stream)."""
+    """Device time of `steps` steps (CUDA events on the launching stream).
+
+    Returns (total_ms, gemm_ms, quant_ms): the per-layer means over the timed
+    steps of the serq_linear and serq_quant_act launches (None without
+    per-launch events)."""
     import torch
     import w4a4_post_quantization_serq_b200 as S
     for _ in range(warmup):
@@ -213,10 +248,12 @@ def time_steps(layers, steps, warmup, pg, per_gemm=True, sampler=None):
         while time.perf_counter() < t_end:
             run_step(layers)
             torch.cuda.synchronize()
-    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in layers] for _ in range(steps)]
+    ev = [[[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in layers] for _ in range(steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(pg)
     torch.cuda.synchronize()
+    switch = sys.getswitchinterval()
+    sys.setswitchinterval(2e-4)  # let the clock sampler thread in while this one launches
     t0 = time.perf_counter()
     start.record()
     for k in range(steps):
@@ -225,12 +262,17 @@ def time_steps(layers, steps, warmup, pg, per_gemm=True, sampler=None):
     torch.cuda.synchronize()
     if sampler is not None:
         sampler.mark(t0, time.perf_counter())
+    sys.setswitchinterval(switch)
     barrier(pg)
     S.serq_device_status()
     total_ms = start.elapsed_time(end)
-    gemm_ms = [sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(steps)) / steps
-               for i in range(len(layers))] if per_gemm else None
-    return total_ms, gemm_ms
+    gemm_ms = quant_ms = None
+    if per_gemm:
+        gemm_ms = [sum(ev[k][i][1].elapsed_time(ev[k][i][2]) for k in range(steps)) / steps
+                   for i in range(len(layers))]
+        quant_ms = [sum(ev[k][i][0].elapsed_time(ev[k][i][1]) for k in range(steps)) / steps
+                    for i in range(len(layers))]
+    return total_ms, gemm_ms, quant_ms
 
 
 def time_e2e(layers, steps, warmup, pg=None):
@@ -503,7 +545,7 @@ def main():
     if not torch.cuda.is_available():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
-    wl = workload(WORKLOAD)
+    wl = workload(args.workload)
     if args.only:
         wl.linears = [l for l in wl.linears if l.name == args.only]
         if not wl.linears:
@@ -512,16 +554,18 @@ def main():
     step_flops = sum(L["flops"] for L in layers)
 
     sampler = ClockSampler(local) if (rank == 0 and not args.no_clocks) else None
-    total_ms, gemm_ms = time_steps(layers, args.steps, args.warmup, pg, sampler=sampler)
+    total_ms, gemm_ms, quant_ms = time_steps(layers, args.steps, args.warmup, pg, sampler=sampler)
     clocks = sampler.stop() if sampler is not None else None
     total_ms = max_over_ranks(pg, total_ms)
     ms_per_step = total_ms / args.steps
     value = whole_job_tops(world, step_flops, ms_per_step)
 
     # dominant kernel: the CTA-pair MXFP4 linear; its largest launch (gate/up,
-    # two thirds of the step's flops) is the roofline's unit
+    # two thirds of the step's flops) is the roofline's unit. The launch lasts
+    # ~0.16 ms inside a ~0.3 ms step, so the burst (not the seconds-long
+    # sustained) GEMM peak is its denominator.
     peaks, peak_src = measured_peaks()
-    fp4_peak = peaks["bf16_tflops_sustained"] * FP4_OVER_BF16
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     dom = max(range(len(layers)), key=lambda i: layers[i]["flops"])
     achieved = layers[dom]["flops"] / (gemm_ms[dom] * 1e-3) / 1e12
     traffic = captured_traffic()
@@ -529,8 +573,10 @@ def main():
                 "frac": achieved / fp4_peak, "traffic": traffic,
                 "kernel": DOMINANT_KERNEL, "launch": layers[dom]["lin"].name,
                 "flops_per_launch": layers[dom]["flops"],
-                "peak_source": f"{peak_src} bf16 sustained {peaks['bf16_tflops_sustained']} TFLOP/s x "
-                               f"{FP4_OVER_BF16:g} (nominal dense FP4/BF16 ratio)",
+                "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
+                               f"{FP4_OVER_BF16:g} (nominal dense FP4/BF16 ratio); of measured",
+                "frac_of_sustained": achieved / (peaks["bf16_tflops_sustained"] * FP4_OVER_BF16),
+                "quant_act": quant_roofline(layers, quant_ms, peaks["hbm_gbs"]),
                 "per_launch_us": {L["lin"].name: round(t * 1e3, 2) for L, t in zip(layers, gemm_ms)},
                 "all_launches_tflops": sum(L["flops"] for L in layers) / (sum(gemm_ms) * 1e-3) / 1e12,
                 "gemm_share_of_step": sum(gemm_ms) / ms_per_step}
@@ -556,7 +602,7 @@ def main():
     if not args.no_extras and rank == 0:
         # SERQ overhead: the same step with r = 0 (plain W4A4)
         layers0 = build_layers(wl, r_override=0)
-        t0, g0 = time_steps(layers0, args.steps, args.warmup, None)
+        t0, g0, _ = time_steps(layers0, args.steps, args.warmup, None)
         del layers0
         torch.cuda.empty_cache()
         line["overhead_vs_r0"] = {"ms_per_step_r0": t0 / args.steps, "step": ms_per_step / (t0 / args.steps) - 1,
@@ -564,11 +610,14 @@ def main():
         # INT4: LLaMA-2-7B q_proj shape
         wl2 = workload("qproj_int4")
         layers2 = build_layers(wl2)
-        t2, g2 = time_steps(layers2, args.steps, args.warmup, None)
+        t2, g2, q2 = time_steps(layers2, args.steps, args.warmup, None)
         f2 = sum(L["flops"] for L in layers2)
         line["int4_qproj"] = {"TOPS": f2 / (t2 / args.steps * 1e-3) / 1e12, "ms_per_step": t2 / args.steps,
                               "serq_linear_us": g2[0] * 1e3,
-                              "frac_of_int8_peak": f2 / (g2[0] * 1e-3) / 1e12 / (peaks["bf16_tflops_sustained"] * 2)}
+                              "frac_of_int8_peak": f2 / (g2[0] * 1e-3) / 1e12 / (peaks["bf16_tflops"] * 2),
+                              "int8_peak_tops": peaks["bf16_tflops"] * 2,
+                              "peak_source": "measured bf16 burst x 2 (nominal dense INT8/BF16 ratio); of measured",
+                              "quant_act": quant_roofline(layers2, q2, peaks["hbm_gbs"])}
         del layers2
     if not args.no_extras and rank == 0:
         dec = bench_decode()

@@ -120,3 +120,14 @@ def test_captured_traffic_tracks_source(tmp_path, monkeypatch):
     fake = dict(rec, kernel="some_other_kernel")
     p.write_text(json.dumps(fake))
     assert bench.captured_traffic() is None
+
+
+def test_quant_act_bytes_closed_form():
+    # LLaMA-3-8B down input, M=2048, K=14336, r=128 (rp=128), MXFP4: read X^ 58.7 MB,
+    # write codes 14.7 MB + 0.13 MB and E8M0 scales 0.92 MB + 8 KB
+    import bench
+    M, K = 2048, 14336
+    assert bench.quant_act_bytes(M, K, 128, "mxfp4") == 2 * M * K + M * K // 2 + M * 64 + M * K // 32 + M * 4
+    # INT4, LLaMA-2-7B q_proj: fp32 per-token scales for the row and the slice
+    assert bench.quant_act_bytes(2048, 4096, 128, "int4") == 2 * 2048 * 4096 + 2048 * 2048 + 2048 * 64 + 8 * 2048
+    assert bench.quant_act_bytes(16, 4096, 0, "int4") == 2 * 16 * 4096 + 16 * 2048 + 4 * 16
