@@ -403,6 +403,77 @@ def serq_forward(X: np.ndarray, W: np.ndarray, r: int, fmt: str,
 
 
 # ---------------------------------------------------------------------------
+# Producers with the offline fold merged in  [notes, Stage 3 "行/列排列离线合并到
+# 权重中"; gist-zh 2.3]: the layer that emits this linear's input writes X^
+# (permuted, divided by s) directly, so the activation quantization can run in
+# the same pass. In a LLaMA block the producers are RMSNorm (before q/k/v and
+# gate/up) and SwiGLU (before down); the pages do not spell these layers out,
+# so they are written here in their standard form.
+# ---------------------------------------------------------------------------
+
+def _f32_of_exact_sum(v: np.ndarray) -> np.float32:
+    """float32 nearest to the exact sum of the float64 values v (ties to even)."""
+    import math
+    v = [float(t) for t in np.asarray(v, dtype=np.float64).reshape(-1)]
+    d = math.fsum(v)                       # the exact sum, correctly rounded to float64
+    f = np.float32(d)                      # float64 -> float32, nearest even
+    if float(f) != d:
+        # d may sit exactly half-way between two float32 values while the exact
+        # sum does not: decide from the sign of the exact remainder
+        lo, hi = (f, np.nextafter(f, np.float32(np.inf))) if float(f) < d else \
+                 (np.nextafter(f, np.float32(-np.inf)), f)
+        mid = (float(lo) + float(hi)) / 2.0    # exact in float64
+        if d == mid:
+            rem = math.fsum(v + [-mid])
+            if rem > 0:
+                f = hi
+            elif rem < 0:
+                f = lo
+    return np.float32(f)
+
+
+def rmsnorm_rstd(H: np.ndarray, eps: float) -> np.ndarray:
+    """rstd[m] = 1 / sqrt(fp32(sum_j H[m,j]^2) / K + eps), each step one fp32 rounding.
+
+    The sum of squares is the exact sum rounded once to fp32 (bf16 inputs square
+    exactly in float64)."""
+    H = np.asarray(H, dtype=F32)
+    M, K = H.shape
+    sq = H.astype(np.float64) ** 2
+    ss = np.array([_f32_of_exact_sum(sq[m]) for m in range(M)], dtype=F32)
+    ms = (ss / F32(K)).astype(F32)
+    v = (ms + F32(eps)).astype(F32)
+    return (F32(1.0) / np.sqrt(v).astype(F32)).astype(F32)
+
+
+def rmsnorm_folded(H: np.ndarray, gamma: np.ndarray, eps: float, perm: np.ndarray,
+                   inv_s: np.ndarray) -> np.ndarray:
+    """RMSNorm producer with the fold:  X^[m, i] = bf16(fp32(H[m, perm[i]] * rstd[m])
+    * fp32(gamma[perm[i]] * inv_s[i])).
+
+    RMSNorm(h) = h / sqrt(mean(h^2) + eps) * gamma; its output channel perm[i]
+    goes to position i divided by s[perm[i]] (1/s folded into gamma)."""
+    H = np.asarray(H, dtype=F32)
+    rstd = rmsnorm_rstd(H, eps)
+    g = (np.asarray(gamma, dtype=F32)[perm] * np.asarray(inv_s, dtype=F32)).astype(F32)
+    t = (H[:, perm] * rstd[:, None]).astype(F32)
+    return bf16_rne((t * g[None, :]).astype(F32))
+
+
+def swiglu_folded(Ygu: np.ndarray, perm: np.ndarray, inv_s: np.ndarray) -> np.ndarray:
+    """SwiGLU producer with the fold, in float64 (no storage rounding):
+    X^[m, i] = silu(g) * u / s, with g = Ygu[m, perm[i]], u = Ygu[m, F + perm[i]],
+    silu(g) = g / (1 + exp(-g)); Ygu = [gate | up] outputs, F columns each."""
+    Y = np.asarray(Ygu, dtype=np.float64)
+    F = Y.shape[1] // 2
+    g = Y[:, :F][:, perm]
+    u = Y[:, F:][:, perm]
+    with np.errstate(over="ignore"):
+        silu = g / (1.0 + np.exp(-g))
+    return silu * u * np.asarray(inv_s, dtype=np.float64)[None, :]
+
+
+# ---------------------------------------------------------------------------
 # canonical packed byte layouts used for bit-exact comparisons
 # ---------------------------------------------------------------------------
 

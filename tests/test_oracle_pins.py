@@ -448,3 +448,71 @@ def test_salient_slice_hand_values(case):
     for c, code in case["codes_slice"].items():
         expect[int(c)] = code
     assert qa.qxs[0].astype(np.int64).tolist() == expect.tolist(), case["why"]
+
+
+# --------------------------------------------------------------------------
+# producers with the fold merged in (Stage 3): RMSNorm and SwiGLU
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", _golden("oracle_hand_cases.json")["exact_sum_to_f32"])
+def test_exact_sum_rounds_once_to_f32(case):
+    got = O._f32_of_exact_sum(np.array(case["v"], np.float64))
+    assert got.dtype == np.float32 and float(got) == case["f32"], case["why"]
+
+
+@pytest.mark.parametrize("case", _golden("oracle_hand_cases.json")["rmsnorm_folded"])
+def test_rmsnorm_folded_hand_values(case):
+    s = np.array(case["s"], np.float32)
+    perm = O.saliency_permutation(s)
+    inv_s = (np.float32(1) / s[perm]).astype(np.float32)
+    H = np.array(case["H"], np.float32)
+    assert O.rmsnorm_rstd(H, case["eps"]).tolist() == case["rstd"]
+    got = O.rmsnorm_folded(H, np.array(case["gamma"], np.float32), case["eps"], perm, inv_s)
+    assert got.tolist() == case["Xhat"], case["why"]
+
+
+def test_rmsnorm_folded_against_textbook_rmsnorm():
+    # h / sqrt(mean(h^2) + eps) * gamma in float64, then permuted and divided by s:
+    # equal to the folded producer up to its fp32 steps and the final bf16 rounding
+    rng = np.random.default_rng(9)
+    M, K, eps = 6, 96, 1e-5
+    H = O.bf16_rne((rng.standard_normal((M, K)) * rng.uniform(0.1, 30, (M, 1))).astype(np.float32))
+    gamma = O.bf16_rne(rng.uniform(0.2, 2.0, K).astype(np.float32))
+    s = np.exp(rng.standard_normal(K)).astype(np.float32)
+    perm = O.saliency_permutation(s)
+    inv_s = (np.float32(1) / s[perm]).astype(np.float32)
+    Hd = H.astype(np.float64)
+    ref = Hd / np.sqrt((Hd ** 2).mean(axis=1, keepdims=True) + eps) * gamma.astype(np.float64)
+    ref = ref[:, perm] / s[perm].astype(np.float64)[None, :]
+    got = O.rmsnorm_folded(H, gamma, eps, perm, inv_s).astype(np.float64)
+    assert np.all(np.abs(got - ref) <= 2.0 ** -8 * np.abs(ref) + 1e-30)
+    # scaling a row by a power of two leaves it unchanged (eps = 0)
+    a = O.rmsnorm_folded(H, gamma, 0.0, perm, inv_s)
+    b = O.rmsnorm_folded((H * np.float32(8)).astype(np.float32), gamma, 0.0, perm, inv_s)
+    assert np.array_equal(a, b)
+    # the fold: position i carries channel perm[i] (a one-hot row lands at perm^-1)
+    one = np.zeros((1, K), np.float32)
+    one[0, 17] = 1.0
+    x = O.rmsnorm_folded(one, np.ones(K, np.float32), 0.0, perm, inv_s)
+    pos = int(np.flatnonzero(x[0])[0])
+    assert perm[pos] == 17 and np.count_nonzero(x) == 1
+
+
+def test_swiglu_folded_closed_forms():
+    g = np.array([0.0, math.log(3.0), -1000.0, 30.0])
+    u = np.array([5.0, 2.0, 1.0, -1.0])
+    Ygu = np.concatenate([g, u])[None, :]
+    perm = np.arange(4)
+    x = O.swiglu_folded(Ygu, perm, np.ones(4))[0]
+    assert x[0] == 0.0                                         # silu(0) = 0
+    assert abs(x[1] - 0.75 * math.log(3.0) * 2.0) < 1e-15     # exp(-ln 3) = 1/3: silu = g / (4/3)
+    assert x[2] == 0.0                                         # exp overflow: g / inf = -0
+    assert abs(x[3] + 30.0 / (1.0 + math.exp(-30.0))) < 1e-12
+    # column mapping: gate channel perm[i] and up channel F + perm[i], divided by s
+    Y = np.array([[1.0, 2.0, 3.0, 10.0, 20.0, 30.0]])
+    perm = np.array([2, 0, 1])
+    inv_s = np.array([0.5, 2.0, 4.0])
+    got = O.swiglu_folded(Y, perm, inv_s)[0]
+    silu = lambda t: t / (1.0 + math.exp(-t))
+    want = [silu(3.0) * 30.0 * 0.5, silu(1.0) * 10.0 * 2.0, silu(2.0) * 20.0 * 4.0]
+    assert np.allclose(got, want, rtol=1e-15, atol=0)
