@@ -239,6 +239,34 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
                            void* xsq, void* xss, serq_stream stream);
 
 /* ------------------------------------------------------------------------
+ * Producers with the fold and the activation quantization fused (reading
+ * notes Stage 3, gist.science/zh 2.3: the permutation and 1/s are merged into
+ * the layer that produces the linear's input). One pass reads the producer's
+ * input and writes serq_quant_act's outputs for X^ (same layouts, same
+ * sizes: serq_act_buffer_sizes(M, w->K, w->r, w->fmt)); X^ itself is not
+ * stored unless `xhat` (bf16 [M][K], may be NULL) asks for a copy.
+ * w is the consuming linear (its perm, 1/s[perm], K, r and format).
+ *
+ * serq_rmsnorm_quant_act: H bf16 [M][K] (original channel order), gamma bf16
+ *   [K], eps >= 0:
+ *     rstd[m] = 1 / sqrt(fp32(sum_j H[m,j]^2) / K + eps)
+ *     X^[m,i] = bf16(fp32(H[m, perm[i]] * rstd[m]) * fp32(gamma[perm[i]] * inv_s[i]))
+ *   Every step is one IEEE fp32 rounding; the sum of squares is accumulated
+ *   in fp64 and rounded once. RMSNorm is the producer of q/k/v and gate/up.
+ * serq_swiglu_quant_act: Ygu bf16 [M][2K] = [gate | up] outputs (original
+ *   channel order):
+ *     X^[m,i] = bf16(fp32(fp32(silu(g) * u) * inv_s[i])), g = Ygu[m, perm[i]],
+ *     u = Ygu[m, K + perm[i]], silu(g) = g / (1 + expf(-g)) in fp32.
+ *   SwiGLU is the producer of down.
+ * Requirements: M >= 1, K <= 32768, 16-byte aligned pointers. Asynchronous.
+ * Errors: EINVAL, EUNSUPPORTED, ECUDA.
+ * ------------------------------------------------------------------------ */
+serq_status serq_rmsnorm_quant_act(const serq_weight* w, const void* H, const void* gamma, float eps, int M,
+                                   void* xq, void* xs, void* xsq, void* xss, void* xhat, serq_stream stream);
+serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, void* xq, void* xs, void* xsq,
+                                  void* xss, void* xhat, serq_stream stream);
+
+/* ------------------------------------------------------------------------
  * The SERQ linear (the "量化推理" formula): one kernel launch computing
  *   MXFP4: Y = bf16( sum over K of X^_q W^_q  +  sum over r of X~_{s,q} Q(R) ),
  *          both block-scaled products accumulated into one fp32 tile;

@@ -11,6 +11,7 @@ from .generators import (  # noqa: F401
     Workload,
     activations,
     bf16_bits,
+    norm_weight,
     round_to_bf16,
     weights,
     workload,

@@ -29,6 +29,7 @@ _STREAM_X = 1
 _STREAM_OUTLIER_IDX = 2
 _STREAM_OUTLIER_MAG = 3
 _STREAM_W = 4
+_STREAM_GAMMA = 5
 
 
 def round_to_bf16(x: np.ndarray) -> np.ndarray:
@@ -71,6 +72,13 @@ def weights(seed: int, K: int, N: int, std: float = 0.02) -> np.ndarray:
     """Weight W (K x N, input channel major) drawn N(0, std^2)."""
     w = np.random.default_rng([seed, _STREAM_W]).standard_normal((K, N), dtype=np.float32)
     return round_to_bf16(w * np.float32(std))
+
+
+def norm_weight(seed: int, K: int, spread: float = 0.2) -> np.ndarray:
+    """RMSNorm weight gamma (K,) drawn 1 + spread * N(0, 1) (a trained norm
+    weight's typical range), rounded to bf16."""
+    g = np.random.default_rng([seed, _STREAM_GAMMA]).standard_normal(K, dtype=np.float32)
+    return round_to_bf16(np.float32(1.0) + np.float32(spread) * g)
 
 
 @dataclasses.dataclass

@@ -19,6 +19,8 @@ from .serq import (  # noqa: F401
     serq_linear_small_m_noalloc,
     serq_prepare,
     serq_quant_act,
+    serq_rmsnorm_quant_act,
+    serq_swiglu_quant_act,
     serq_selftest_wait,
     serq_version,
     serq_weight_create_from_host,

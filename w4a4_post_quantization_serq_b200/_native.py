@@ -51,6 +51,10 @@ _SIGNATURES = {
     "serq_act_buffer_sizes": (c_int, [c_int, c_int, c_int, c_int, ctypes.POINTER(ActSizes)]),
     "serq_quant_act": (c_int, [c_void_p, c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                c_void_p]),
+    "serq_rmsnorm_quant_act": (c_int, [c_void_p, c_void_p, c_void_p, ctypes.c_float, c_int, c_void_p, c_void_p,
+                                       c_void_p, c_void_p, c_void_p, c_void_p]),
+    "serq_swiglu_quant_act": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                      c_void_p]),
     "serq_linear": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p]),
     "serq_linear_small_m_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,

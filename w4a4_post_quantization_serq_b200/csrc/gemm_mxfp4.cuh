@@ -57,11 +57,6 @@ struct MxParams {
     __nv_bfloat16* Y;
 };
 
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
 __global__ void __launch_bounds__(mx::THREADS, 1)
 serq_linear_mxfp4_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                          const __grid_constant__ CUtensorMap tm_ar, const __grid_constant__ CUtensorMap tm_br,

@@ -395,6 +395,12 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
            | (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// Two floats -> two bf16 (round to nearest even) in one word, `lo` in the low half.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const uint32_t*>(&h);
+}
+
 __device__ __forceinline__ uint32_t elect_one_lane() {
     return (threadIdx.x & 31) == 0;
 }

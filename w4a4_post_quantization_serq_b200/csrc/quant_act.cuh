@@ -98,23 +98,29 @@ __device__ __forceinline__ float block_max2(float& a, float& b, float* red) {
     return a;
 }
 
-// One CTA per token row. MAXC = 16-byte chunks held per thread (K <= 8 * 256 * MAXC).
-template <int MAXC>
-__global__ void __launch_bounds__(kQuantThreads)
-quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
-                      float* __restrict__ xs, uint32_t* __restrict__ xsq, float* __restrict__ xss) {
-    __shared__ float red[64];
-    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
-    const int m = blockIdx.x;
+// ---------------------------------------------------------------- row quantizers
+// A "chunk source" yields the row's values eight at a time as packed bf16
+// (chunk c = positions 8c .. 8c+7 of X^[m, :]); the quantizers below turn a
+// row into serq_quant_act's outputs. The plain quantizer reads X^ from global
+// memory; the fused producers compute X^ on the fly (producer.cuh).
+struct SrcBf16Row {
+    const uint4* row;
+    __device__ __forceinline__ uint4 chunk(int c) const { return __ldg(row + c); }
+};
+
+// INT4, one CTA per row. MAXC = 16-byte chunks held per thread (K <= 8 * 256 * MAXC).
+template <int MAXC, class Src>
+__device__ __forceinline__ void quant_row_int4(const Src& src, int m, int K, int r, int rp, uint32_t* __restrict__ xq,
+                                               float* __restrict__ xs, uint32_t* __restrict__ xsq,
+                                               float* __restrict__ xss, float* red) {
     const int nchunk = K >> 3;
-    const uint4* row = X + static_cast<size_t>(m) * nchunk;
     uint4 v[MAXC];
     float amax = 0.0f, amax_s = 0.0f;
 #pragma unroll
     for (int j = 0; j < MAXC; ++j) {
         const int c = threadIdx.x + j * kQuantThreads;
         if (c < nchunk) {
-            v[j] = __ldg(row + c);
+            v[j] = src.chunk(c);
             float f[8];
             bf16x8_to_f32(v[j], f);
 #pragma unroll
@@ -154,25 +160,22 @@ quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_
     }
 }
 
-// One CTA per token row; four consecutive threads share one 32-element block.
-__global__ void __launch_bounds__(kQuantThreads)
-quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
-                       uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
-                       uint8_t* __restrict__ xss_atoms) {
-    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
-    const int m = blockIdx.x;
+// MXFP4, one CTA per row; four consecutive threads share one 32-element block.
+template <class Src>
+__device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, int r, int rp,
+                                                uint32_t* __restrict__ xq, uint8_t* __restrict__ xs_atoms,
+                                                uint32_t* __restrict__ xsq, uint8_t* __restrict__ xss_atoms) {
     const int nchunk = K >> 3;
     const int atoms_k = (K / 32 + 3) / 4;
     const int nchunk_s = rp >> 3;
     const int atoms_s = (rp / 32 + 3) / 4;
-    const uint4* row = X + static_cast<size_t>(m) * nchunk;
     const int iters = (nchunk + kQuantThreads - 1) / kQuantThreads;
     for (int j = 0; j < iters; ++j) {
         const int c = threadIdx.x + j * kQuantThreads;
         const bool valid = c < nchunk;
         float f[8];
         if (valid) {
-            bf16x8_to_f32(__ldg(row + c), f);
+            bf16x8_to_f32(src.chunk(c), f);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = 0.0f;
@@ -208,6 +211,28 @@ quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32
                 xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
         }
     }
+}
+
+// serq_quant_act: one CTA per token row of X^ (bf16, row-major).
+template <int MAXC>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
+                      float* __restrict__ xs, uint32_t* __restrict__ xsq, float* __restrict__ xss) {
+    __shared__ float red[64];
+    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
+    const int m = blockIdx.x;
+    const SrcBf16Row src{X + static_cast<size_t>(m) * (K >> 3)};
+    quant_row_int4<MAXC>(src, m, K, r, rp, xq, xs, xsq, xss, red);
+}
+
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
+                       uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
+                       uint8_t* __restrict__ xss_atoms) {
+    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
+    const int m = blockIdx.x;
+    const SrcBf16Row src{X + static_cast<size_t>(m) * (K >> 3)};
+    quant_row_mxfp4(src, m, K, r, rp, xq, xs_atoms, xsq, xss_atoms);
 }
 
 }  // namespace serq

@@ -18,6 +18,7 @@
 
 #include "ptx.cuh"
 #include "quant_act.cuh"
+#include "producer.cuh"
 #include "prepare.cuh"
 #include "gemm_mxfp4.cuh"
 #include "gemm_int4.cuh"
@@ -72,6 +73,7 @@ struct DeviceInfo {
     bool smem_set_i4 = false;
     bool smem_set_mxd = false;
     bool smem_set_mxp = false;
+    bool smem_set_prod = false;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
 };
 
@@ -901,6 +903,96 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
     }
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
+}
+
+}  // extern "C"
+
+namespace {
+
+template <int KIND, int FMT, int MAXC>
+serq_status producer_setup_one() {
+    SERQ_CUDA(cudaFuncSetAttribute(producer_quant_kernel<KIND, FMT, MAXC>,
+                                   cudaFuncAttributeMaxDynamicSharedMemorySize, 4 * 32768));
+    return SERQ_OK;
+}
+
+serq_status producer_setup(DeviceInfo* info) {
+    if (info->smem_set_prod) return SERQ_OK;
+    serq_status st = producer_setup_one<0, 0, 8>();
+    if (!st) st = producer_setup_one<0, 0, 16>();
+    if (!st) st = producer_setup_one<0, 1, 1>();
+    if (!st) st = producer_setup_one<1, 0, 8>();
+    if (!st) st = producer_setup_one<1, 0, 16>();
+    if (!st) st = producer_setup_one<1, 1, 1>();
+    if (!st) info->smem_set_prod = true;
+    return st;
+}
+
+// Shared checks and launch of the fused producer + quantization kernels.
+serq_status producer_launch(int kind, const serq_weight* w, const void* in, const void* gamma, float eps, int M,
+                            void* xq, void* xs, void* xsq, void* xss, void* xhat, serq_stream stream) {
+    if (w == nullptr || in == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    if (M < 1) return fail(SERQ_EINVAL, "M must be >= 1");
+    if (kind == 0 && (gamma == nullptr || !aligned16(gamma))) return fail(SERQ_EINVAL, "gamma must be a 16-byte aligned pointer");
+    if (kind == 0 && !(eps >= 0.0f && std::isfinite(eps))) return fail(SERQ_EINVAL, "eps must be finite and >= 0");
+    if (xq == nullptr || xs == nullptr) return fail(SERQ_EINVAL, "NULL output");
+    if (w->rp > 0 && (xsq == nullptr || xss == nullptr)) return fail(SERQ_EINVAL, "r > 0 needs xsq and xss");
+    if (!aligned16(in) || !aligned16(xq) || !aligned16(xs) || !aligned16(xhat) ||
+        (w->rp > 0 && (!aligned16(xsq) || !aligned16(xss))))
+        return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    if (dev != w->device) return fail(SERQ_EINVAL, "weight lives on device %d, current device is %d", w->device, dev);
+    if (serq_status st = producer_setup(info)) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    ProducerParams p;
+    p.K = w->K;
+    p.r = w->r;
+    p.rp = w->rp;
+    p.perm = w->perm;
+    p.inv_s = w->inv_s;
+    p.gamma = static_cast<const __nv_bfloat16*>(gamma);
+    p.eps = eps;
+    p.xq = xq;
+    p.xs = xs;
+    p.xsq = xsq;
+    p.xss = xss;
+    p.xhat = static_cast<__nv_bfloat16*>(xhat);
+    const uint4* src = static_cast<const uint4*>(in);
+    const size_t smem = static_cast<size_t>(w->K) * (kind == 0 ? 2 : 4);
+    const bool wide = w->K > 16384;
+    if (kind == 0) {
+        if (w->fmt == SERQ_FMT_MXFP4)
+            producer_quant_kernel<0, 1, 1><<<M, kQuantThreads, smem, cs>>>(src, p);
+        else if (wide)
+            producer_quant_kernel<0, 0, 16><<<M, kQuantThreads, smem, cs>>>(src, p);
+        else
+            producer_quant_kernel<0, 0, 8><<<M, kQuantThreads, smem, cs>>>(src, p);
+    } else {
+        if (w->fmt == SERQ_FMT_MXFP4)
+            producer_quant_kernel<1, 1, 1><<<M, kQuantThreads, smem, cs>>>(src, p);
+        else if (wide)
+            producer_quant_kernel<1, 0, 16><<<M, kQuantThreads, smem, cs>>>(src, p);
+        else
+            producer_quant_kernel<1, 0, 8><<<M, kQuantThreads, smem, cs>>>(src, p);
+    }
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+serq_status serq_rmsnorm_quant_act(const serq_weight* w, const void* H, const void* gamma, float eps, int M, void* xq,
+                                   void* xs, void* xsq, void* xss, void* xhat, serq_stream stream) {
+    return producer_launch(0, w, H, gamma, eps, M, xq, xs, xsq, xss, xhat, stream);
+}
+
+serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, void* xq, void* xs, void* xsq,
+                                  void* xss, void* xhat, serq_stream stream) {
+    return producer_launch(1, w, Ygu, nullptr, 0.0f, M, xq, xs, xsq, xss, xhat, stream);
 }
 
 serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void* xs, const void* xsq,

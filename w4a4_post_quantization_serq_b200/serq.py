@@ -238,6 +238,30 @@ def serq_quant_act(Xhat: torch.Tensor, r: int, fmt, out: Optional[QuantAct] = No
     return out
 
 
+def serq_rmsnorm_quant_act(w: SerqWeight, H: torch.Tensor, gamma: torch.Tensor, eps: float,
+                           out: Optional[QuantAct] = None, xhat: Optional[torch.Tensor] = None,
+                           stream=None) -> QuantAct:
+    """RMSNorm producer with w's fold and the activation quantization in one pass (H: bf16 M x K)."""
+    M = H.shape[0]
+    if out is None:
+        out = alloc_act(M, w.K, w.r, w.fmt, H.device)
+    N.check(N.load().serq_rmsnorm_quant_act(w.handle, _ptr(H), _ptr(gamma), float(eps), M, _ptr(out.xq),
+                                            _ptr(out.xs), _ptr(out.xsq), _ptr(out.xss), _ptr(xhat),
+                                            _stream(stream)))
+    return out
+
+
+def serq_swiglu_quant_act(w: SerqWeight, Ygu: torch.Tensor, out: Optional[QuantAct] = None,
+                          xhat: Optional[torch.Tensor] = None, stream=None) -> QuantAct:
+    """SwiGLU producer ([gate | up], bf16 M x 2K) with w's fold and the quantization in one pass."""
+    M = Ygu.shape[0]
+    if out is None:
+        out = alloc_act(M, w.K, w.r, w.fmt, Ygu.device)
+    N.check(N.load().serq_swiglu_quant_act(w.handle, _ptr(Ygu), M, _ptr(out.xq), _ptr(out.xs), _ptr(out.xsq),
+                                           _ptr(out.xss), _ptr(xhat), _stream(stream)))
+    return out
+
+
 def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
                 acc_dbg: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Y = X^_q W^_q + X~_{s,q} Q(R), bf16 M x N, in one kernel launch."""
