@@ -13,6 +13,7 @@ Sources (cited by page title and section):
   [gist-zh] technical summary (gist.science/zh): 2.1 静态激活展平,
             2.2 显著性感知误差重建, 2.3 离线权重置换, 3 主要贡献.
   [gist-pt] resumo técnico (gist.science/pt): 2. Metodologia items 1-3.
+  [abstract] fugumt.com page with the arXiv abstract: W4A8 and W4A4 settings.
   [MX]      OCP Microscaling Formats (MX) Specification v1.0 — the pages only
             name MXFP4; its element (E2M1) and shared-scale (E8M0) rules come
             from this public specification.
@@ -46,10 +47,12 @@ import numpy as np
 
 F32 = np.float32
 INT4_QMAX = 7                       # 2^(n-1) - 1 with n = 4  [notes, 基础量化]
+INT8_QMAX = 127                     # n = 8: the activations of the W4A8 setting [abstract]
 MX_BLOCK = 32                       # elements sharing one E8M0 scale  [MX]
 E2M1_EMAX = 2                       # exponent of the largest E2M1 normal (6 = 1.5 * 2^2)  [MX]
 E8M0_BIAS = 127                     # [MX]
 E2M1_GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])  # magnitudes of codes 0..7  [MX]
+INT_WEIGHT_FORMATS = ("int4", "w4a8")  # INT4 weights; activations INT4 or INT8
 
 
 # ---------------------------------------------------------------------------
@@ -66,31 +69,52 @@ def bf16_rne(x: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# A1: symmetric absmax INT4 quantizer  [notes, 基础量化]
+# A1: symmetric absmax n-bit integer quantizer  [notes, 基础量化]
 #     X_q = clip(round(X / s)),  s = max|X| / (2^(n-1) - 1)
+# n = 4 everywhere in W4A4; n = 8 for the activations of W4A8 [abstract].
 # ---------------------------------------------------------------------------
 
-def int4_scale(absmax: np.ndarray) -> np.ndarray:
-    """s = fp32(max|X| / 7)."""
-    return (np.asarray(absmax, dtype=F32) / F32(INT4_QMAX)).astype(F32)
+def int_scale(absmax: np.ndarray, qmax: int) -> np.ndarray:
+    """s = fp32(max|X| / qmax), qmax = 2^(n-1) - 1."""
+    return (np.asarray(absmax, dtype=F32) / F32(qmax)).astype(F32)
 
 
-def int4_codes(x: np.ndarray, s: np.ndarray) -> np.ndarray:
-    """q = clip(rne(fp32(x / s)), -7, 7); all-zero codes where s == 0."""
+def int_codes(x: np.ndarray, s: np.ndarray, qmax: int) -> np.ndarray:
+    """q = clip(rne(fp32(x / s)), -qmax, qmax); all-zero codes where s == 0."""
     x = np.asarray(x, dtype=F32)
     s = np.asarray(s, dtype=F32)
     with np.errstate(divide="ignore", invalid="ignore"):
         v = (x / s).astype(F32)
     q = np.rint(v)
     q = np.where(s > 0, q, 0.0)
-    return np.clip(q, -INT4_QMAX, INT4_QMAX).astype(np.int8)
+    return np.clip(q, -qmax, qmax).astype(np.int8)
+
+
+def quantize_int(x: np.ndarray, axis: int, qmax: int):
+    """Per-slice symmetric n-bit along ``axis``: returns (codes int8, scale fp32)."""
+    x = np.asarray(x, dtype=F32)
+    s = int_scale(np.max(np.abs(x), axis=axis, keepdims=True), qmax)
+    return int_codes(x, s, qmax), np.squeeze(s, axis=axis)
+
+
+def int4_scale(absmax: np.ndarray) -> np.ndarray:
+    """s = fp32(max|X| / 7)."""
+    return int_scale(absmax, INT4_QMAX)
+
+
+def int4_codes(x: np.ndarray, s: np.ndarray) -> np.ndarray:
+    """q = clip(rne(fp32(x / s)), -7, 7); all-zero codes where s == 0."""
+    return int_codes(x, s, INT4_QMAX)
 
 
 def quantize_int4(x: np.ndarray, axis: int):
     """Per-slice symmetric INT4 along ``axis``: returns (codes int8, scale fp32)."""
-    x = np.asarray(x, dtype=F32)
-    s = int4_scale(np.max(np.abs(x), axis=axis, keepdims=True))
-    return int4_codes(x, s), np.squeeze(s, axis=axis)
+    return quantize_int(x, axis, INT4_QMAX)
+
+
+def quantize_int8(x: np.ndarray, axis: int):
+    """Per-slice symmetric INT8 along ``axis`` (codes in [-127, 127])."""
+    return quantize_int(x, axis, INT8_QMAX)
 
 
 # ---------------------------------------------------------------------------
@@ -244,13 +268,13 @@ class Prepared:
 
     def deq_w(self) -> np.ndarray:
         """Dequantized main weight, [N, K] float64."""
-        if self.fmt == "int4":
+        if self.fmt in INT_WEIGHT_FORMATS:
             return self.qw.astype(np.float64) * self.sw.astype(np.float64)[:, None]
         return mxfp4_dequant(self.qw, self.Ew)
 
     def deq_R(self) -> np.ndarray:
         """Dequantized residual, [N, r] float64."""
-        if self.fmt == "int4":
+        if self.fmt in INT_WEIGHT_FORMATS:
             return self.qR.astype(np.float64) * self.sR.astype(np.float64)[:, None]
         return mxfp4_dequant(self.qR, self.ER)[:, : self.r]
 
@@ -268,11 +292,14 @@ def prepare(W: np.ndarray, r: int, fmt: str, act_absmax: Optional[np.ndarray] = 
        weight quantization                                      [notes, Stage 2]
     6. Q(R): 4-bit, INT4 per output channel, MXFP4 per 32 along r  [gist-zh 2.2]
 
+    fmt "w4a8" prepares the weight exactly as "int4" (4-bit weights, R 4-bit);
+    only its activations differ (8-bit, see quant_act)            [abstract]
+
     ``columns`` restricts steps 3-6 to a subset of output channels (the
     quantization of each output channel is independent of the others); s and
     perm always use all of W.
     """
-    assert fmt in ("int4", "mxfp4")
+    assert fmt in ("int4", "w4a8", "mxfp4")
     W = np.asarray(W, dtype=F32)
     K, N = W.shape
     assert 0 <= r <= K
@@ -285,7 +312,7 @@ def prepare(W: np.ndarray, r: int, fmt: str, act_absmax: Optional[np.ndarray] = 
     Wc = W if columns is None else W[:, columns]
     W_hat = fold_weight(Wc, s, perm)                       # [K, Nc] fp32
     Wt = np.ascontiguousarray(W_hat.T)                     # [Nc, K]
-    if fmt == "int4":
+    if fmt in INT_WEIGHT_FORMATS:
         qw, sw = quantize_int4(Wt, axis=1)                 # per output channel over K
         deq_s = (qw[:, :r].astype(F32) * sw[:, None]).astype(F32)
         R = (Wt[:, :r] - deq_s).astype(F32)                # [Nc, r]
@@ -327,12 +354,12 @@ class QuantAct:
     Exs: Optional[np.ndarray]  # MXFP4: int32 [M, nbr]
 
     def deq_x(self) -> np.ndarray:
-        if self.fmt == "int4":
+        if self.fmt in INT_WEIGHT_FORMATS:
             return self.qx.astype(np.float64) * self.sx.astype(np.float64)[:, None]
         return mxfp4_dequant(self.qx, self.Ex)
 
     def deq_xs(self) -> np.ndarray:
-        if self.fmt == "int4":
+        if self.fmt in INT_WEIGHT_FORMATS:
             return self.qxs.astype(np.float64) * self.sxs.astype(np.float64)[:, None]
         return mxfp4_dequant(self.qxs, self.Exs)[:, : self.r]
 
@@ -341,10 +368,11 @@ def quant_act(Xhat: np.ndarray, r: int, fmt: str) -> QuantAct:
     """Quantize X^ per token and, under its own scale, the salient slice X^[:, :r]."""
     X = np.asarray(Xhat, dtype=F32)
     M, K = X.shape
-    if fmt == "int4":
-        qx, sx = quantize_int4(X, axis=1)
+    if fmt in INT_WEIGHT_FORMATS:
+        qmax = INT8_QMAX if fmt == "w4a8" else INT4_QMAX
+        qx, sx = quantize_int(X, 1, qmax)
         if r > 0:
-            qxs, sxs = quantize_int4(X[:, :r], axis=1)
+            qxs, sxs = quantize_int(X[:, :r], 1, qmax)
         else:
             qxs, sxs = np.zeros((M, 0), np.int8), np.zeros(M, F32)
         return QuantAct(fmt, r, qx, sx, None, qxs, sxs, None)
@@ -362,7 +390,7 @@ def quant_act(Xhat: np.ndarray, r: int, fmt: str) -> QuantAct:
 
 def _exact_int_matmul(a: np.ndarray, b: np.ndarray) -> np.ndarray:
     """Integer matmul a[M,K] @ b[K,N] via float64 (exact: |partial sums| << 2^53)."""
-    assert a.shape[1] * 49 < 2 ** 52
+    assert a.shape[1] * 127 * 7 < 2 ** 52
     c = np.asarray(a, dtype=np.float64) @ np.asarray(b, dtype=np.float64)
     ci = c.astype(np.int64)
     assert np.array_equal(ci, c)
@@ -379,7 +407,7 @@ class LinearOut:
 def linear(prep: Prepared, qa: QuantAct) -> LinearOut:
     """Main 4-bit product plus the single residual product, no intermediate quantization."""
     assert prep.fmt == qa.fmt and prep.r == qa.r
-    if prep.fmt == "int4":
+    if prep.fmt in INT_WEIGHT_FORMATS:
         acc1 = _exact_int_matmul(qa.qx, prep.qw.T)
         acc2 = _exact_int_matmul(qa.qxs, prep.qR.T) if prep.r > 0 else np.zeros_like(acc1)
         assert np.abs(acc1).max(initial=0) < 2 ** 31 and np.abs(acc2).max(initial=0) < 2 ** 31

@@ -516,3 +516,64 @@ def test_swiglu_folded_closed_forms():
     silu = lambda t: t / (1.0 + math.exp(-t))
     want = [silu(3.0) * 30.0 * 0.5, silu(1.0) * 10.0 * 2.0, silu(2.0) * 20.0 * 4.0]
     assert np.allclose(got, want, rtol=1e-15, atol=0)
+
+
+# --------------------------------------------------------------------------
+# W4A8 (the abstract's second setting): INT4 weights and residual, INT8
+# activations and salient slice, the same runtime formula
+# --------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", _golden("quantizer_hand_cases.json")["int8"])
+def test_int8_hand_cases(case):
+    q, s = O.quantize_int8(np.array([case["x"]], dtype=np.float32), axis=1)
+    assert float(s[0]) == case["scale"]
+    assert q[0].tolist() == case["codes"]
+
+
+def test_w4a8_grid_and_weight_equal_to_int4():
+    X = activations(81, 16, 128, 3, "lognormal", 50.0)
+    W = weights(82, 128, 24)
+    p8, Xh, qa, out = O.serq_forward(X, W, 32, "w4a8")
+    p4 = O.prepare(W, 32, "int4", act_absmax=O.calib_absmax(X))
+    # the weight side is the INT4 preparation, bit for bit
+    for k in ("perm", "qw", "sw", "qR", "sR"):
+        assert np.array_equal(getattr(p8, k), getattr(p4, k)), k
+    assert qa.qx.min() >= -127 and qa.qx.max() <= 127 and qa.qx.dtype == np.int8
+    assert np.abs(qa.qx).max() == 127                       # each row's absmax maps to 127
+    sx = np.max(np.abs(Xh), axis=1) / np.float32(127)
+    assert np.array_equal(qa.sx, sx.astype(np.float32))
+
+
+def test_w4a8_r0_is_plain_w4a8_scalar_loops():
+    X = activations(83, 4, 64, 2, "const", 30.0)
+    W = weights(84, 64, 8)
+    prep, Xh, qa, out = O.serq_forward(X, W, 0, "w4a8")
+    M, K = Xh.shape
+    N = W.shape[1]
+    Wh = prep.W_hat
+    for m in range(M):
+        sx = np.float32(max(abs(float(v)) for v in Xh[m])) / np.float32(127)
+        for n in range(N):
+            sw = np.float32(max(abs(float(Wh[k, n])) for k in range(K))) / np.float32(7)
+            acc = 0
+            for k in range(K):
+                qx = max(-127, min(127, round(float(np.float32(Xh[m, k]) / sx))))
+                qw = max(-7, min(7, round(float(np.float32(Wh[k, n]) / sw))))
+                acc += qx * qw
+            assert out.acc1[m, n] == acc
+            assert out.Y[m, n] == acc * float(sx) * float(sw)
+
+
+def test_w4a8_brute_force_and_more_accurate_than_w4a4():
+    wl = workload("tiny_int4")
+    lin = wl.linears[0]
+    X, W = lin.X(wl.M), lin.W()
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    errs = {}
+    for fmt in ("int4", "w4a8"):
+        prep, Xh, qa, out = O.serq_forward(X, W, 16, fmt)
+        # dequantize every operand, multiply with a plain matmul: same Y
+        Yb = qa.deq_x() @ prep.deq_w().T + qa.deq_xs() @ prep.deq_R().T
+        assert np.max(np.abs(Yb - out.Y)) <= 1e-12 * np.max(np.abs(Yb))
+        errs[fmt] = np.linalg.norm(out.Y - ref)
+    assert errs["w4a8"] < errs["int4"]
