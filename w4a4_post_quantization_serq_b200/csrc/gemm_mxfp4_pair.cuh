@@ -18,12 +18,15 @@
 // single hop.
 //
 // Scale atoms reach tensor memory by tcgen05.cp, which the tensor pipe runs
-// in order with the MMAs: each copy costs pipe time between K-tiles, so the
-// weight scales come in a prepared "wide" layout (each 512 B atom repeated
-// four times, the two 128-row halves side by side, 4 KB per atom pair) that
-// one .128x256b copy moves per K-atom instead of two .32x128b.warpx4 copies.
-// The activation scales (written per call by serq_quant_act in the canonical
-// layout) keep the narrow copies: 4 copies per K-tile instead of 6.
+// in order with the MMAs: each copy costs pipe time between K-tiles, so every
+// scale tile is copied in the "wide" form one .128x256b copy moves (each
+// 512 B atom repeated four times so that every 32-lane quarter of tensor
+// memory gets its rows, two atoms side by side): 3 copies per K-tile instead
+// of 6 narrow .32x128b.warpx4 ones. The weight scales are stored wide at
+// prepare (each 4 KB piece: one K-atom, both 128-row halves of the pair
+// tile). The activation scales arrive per call in the canonical atom layout;
+// four 3-D TMA loads of the K-tile's two atoms (1 KB, served from L2 after the
+// first) build their 4 KB wide tile in shared memory.
 //
 // Epilogue stores: a thread holds one output row, so storing straight from
 // registers would make every warp store touch 32 rows with 16 B each (half
@@ -55,10 +58,10 @@ constexpr int BN = 256;                       // output channels per pair tile
 constexpr int BN_HALF = 128;                  // rows of B per CTA
 constexpr int BK_BYTES = 128;
 constexpr int BK = 256;
-constexpr int STAGES = 5;
+constexpr int STAGES = 4;
 constexpr int A_BYTES = BM * BK_BYTES;        // 16 KB
 constexpr int B_BYTES = BN_HALF * BK_BYTES;   // 16 KB
-constexpr int SFA_BYTES = 2 * 512;            // own 128 rows x 8 scales
+constexpr int SFA_BYTES = 4 * 2 * 512;        // own 128 rows x 8 scales, wide (4 replicas of 2 atoms)
 constexpr int SFB_BYTES = 2 * 4096;           // all 256 rows x 8 scales, wide layout (2 atom pairs)
 constexpr uint32_t STAGE_TX = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // bytes one CTA loads per stage
 constexpr int NUM_EPI_WARPS = 8;
@@ -85,9 +88,11 @@ struct MxPairParams {
     __nv_bfloat16* Y;
 };
 
-// Scale tensor maps, arrays viewed as rows of 256 B (rows past the end read as
-// zeros): activation atoms with box 256 x 4 (two 512 B atoms), wide weight
-// scales with box 256 x 32 (two 4 KB atom pairs).
+// Scale tensor maps (reads past the end give zeros). Activation atoms as a
+// 3-D view (x: 128 bytes, atom: stride 512, piece: stride 128) with box
+// 128 x 2 x 4: one load gives both atoms of a K-tile as 32 row groups of 128 B
+// in wide order (piece-major, then atom); wide weight scales as rows of 256 B
+// with box 256 x 32 (two 4 KB pieces).
 struct MxPairScaleMaps {
     CUtensorMap sfa, sfb, sfa_r, sfb_r;
 };
@@ -181,9 +186,11 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                     tma_load_2d_pair(sA + s * A_BYTES, res ? &tm_ar : &tm_a, bar, kk * BK_BYTES, a_rowblk * BM);
                     tma_load_2d_pair(sB + s * B_BYTES, res ? &tm_br : &tm_b, bar, kk * BK_BYTES,
                                      n_blk * BN + static_cast<int>(rank) * BN_HALF);
-                    // scale atoms (2 per K-tile) as rows of 256 B
-                    tma_load_2d_pair(sSFA + s * SFA_BYTES, res ? &sf.sfa_r : &sf.sfa, bar, 0,
-                                     (a_rowblk * atoms + 2 * kk) * 2);
+                    // activation scale atoms (2 per K-tile), four replicas = the wide tile
+#pragma unroll
+                    for (int rep = 0; rep < 4; ++rep)
+                        tma_load_3d_pair(sSFA + s * SFA_BYTES + rep * 1024, res ? &sf.sfa_r : &sf.sfa, bar, 0,
+                                         a_rowblk * atoms + 2 * kk, 0);
                     tma_load_2d_pair(sSFB + s * SFB_BYTES, res ? &sf.sfb_r : &sf.sfb, bar, 0,
                                      (n_blk * atoms + 2 * kk) * 16);
                     if (++s == STAGES) {
@@ -234,10 +241,8 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
                     const uint32_t b_base = smem_u32(sB + s * B_BYTES);
                     const uint32_t sfa_base = smem_u32(sSFA + s * SFA_BYTES);
                     const uint32_t sfb_base = smem_u32(sSFB + s * SFB_BYTES);
-                    for (int j = 0; j < na; ++j) {
-                        tc_cp_32x128b_warpx4_pair(tmem + TMEM_SFA + 4 * j, sdesc_sf_atom(sfa_base + 512 * j));
-                        tc_cp_128x256b_pair(tmem + TMEM_SFB + 8 * j, sdesc_sf_wide(sfb_base + 4096 * j));
-                    }
+                    tc_cp_128x256b_pair(tmem + TMEM_SFA, sdesc_sf_wide(sfa_base));
+                    for (int j = 0; j < na; ++j) tc_cp_128x256b_pair(tmem + TMEM_SFB + 8 * j, sdesc_sf_wide(sfb_base + 4096 * j));
                     for (int st = 0; st < steps; ++st) {
                         tc_mma_mxf4_pair(tmem + acc_col, sdesc_kmajor_sw128(a_base + 32 * st),
                                          sdesc_kmajor_sw128(b_base + 32 * st), (st & 1) ? id_odd : id_even,

@@ -213,6 +213,72 @@ __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, in
     }
 }
 
+// MXFP4 serq_quant_act as a flat stream over all of X^: an MX block (32
+// values, four 16-byte chunks) never needs more than its own row segment, so
+// the grid walks the M x K/8 chunks directly. Each warp covers QF_UNROLL groups
+// of 32 consecutive chunks per pass (the four chunks of a block in four
+// consecutive lanes), with all its loads issued before any is used.
+constexpr int QF_UNROLL = 4;
+
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int M, int K, int r, int rp, uint32_t* __restrict__ xq,
+                            uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
+                            uint8_t* __restrict__ xss_atoms) {
+    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
+    const int nchunk = K >> 3;                 // chunks per row (a multiple of 16)
+    const int nchunk_s = rp >> 3;
+    const int atoms_k = (K / 32 + 3) / 4;
+    const int atoms_s = (rp / 32 + 3) / 4;
+    const long long total = static_cast<long long>(M) * nchunk;
+    const int lane = threadIdx.x & 31;
+    const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
+    for (long long base = warp_id * (32 * QF_UNROLL); base < total; base += n_warps * (32 * QF_UNROLL)) {
+        uint4 v[QF_UNROLL];
+#pragma unroll
+        for (int u = 0; u < QF_UNROLL; ++u) {
+            const long long c = base + u * 32 + lane;
+            v[u] = c < total ? __ldcs(X + c) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int u = 0; u < QF_UNROLL; ++u) {
+            const long long c = base + u * 32 + lane;
+            const bool valid = c < total;          // uniform over each group of four lanes
+            const int m = valid ? static_cast<int>(c / nchunk) : 0;
+            const int cc = valid ? static_cast<int>(c - static_cast<long long>(m) * nchunk) : 0;
+            float f[8];
+            bf16x8_to_f32(v[u], f);
+            float a = 0.0f, as = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                a = fmaxf(a, fabsf(f[e]));
+                if (cc * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
+            }
+            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+            if (!valid) continue;
+            const int blk = cc >> 2;
+            const int E = mx_exponent(a);
+            const float inv = mx_inv_scale(E);
+            float g[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
+            xq[c] = e2m1x8(g);
+            if ((lane & 3) == 0) xs_atoms[sf_atom_offset(m, blk, atoms_k)] = static_cast<uint8_t>(E + 127);
+            if (cc < nchunk_s) {
+                const int Es = mx_exponent(as);
+                const float invs = mx_inv_scale(Es);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) g[e] = (cc * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+                xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
+                if ((lane & 3) == 0) xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
+            }
+        }
+    }
+}
+
 // serq_quant_act: one CTA per token row of X^ (bf16, row-major).
 template <int MAXC>
 __global__ void __launch_bounds__(kQuantThreads)
@@ -225,14 +291,5 @@ quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_
     quant_row_int4<MAXC>(src, m, K, r, rp, xq, xs, xsq, xss, red);
 }
 
-__global__ void __launch_bounds__(kQuantThreads)
-quant_act_mxfp4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
-                       uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
-                       uint8_t* __restrict__ xss_atoms) {
-    pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
-    const int m = blockIdx.x;
-    const SrcBf16Row src{X + static_cast<size_t>(m) * (K >> 3)};
-    quant_row_mxfp4(src, m, K, r, rp, xq, xs_atoms, xsq, xss_atoms);
-}
 
 }  // namespace serq

@@ -156,10 +156,22 @@ EncodeTiledFn encode_fn() {
 serq_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
                      uint32_t box_rows, bool swizzle128);
 
-// MXFP4 scale-atom array (a multiple of 512 B) as rows of 256 B; a box is two
-// atoms (256 x 4). Rows past the end read as zeros.
-serq_status make_scale_map(CUtensorMap* map, const void* base, size_t bytes) {
-    return make_map(map, base, 256, bytes / 256, 256, 4, false);
+// MXFP4 activation scale atoms (`bytes`, a multiple of 512) as the 3-D view
+// the CTA-pair kernel reads its wide scale tiles through: x = byte within a
+// 128-byte piece, y = atom (stride 512), z = piece of the atom (stride 128);
+// a box of 128 x 2 x 4 is a K-tile's two atoms, pieces outermost.
+serq_status make_sfa_wide_map(CUtensorMap* map, const void* base, size_t bytes) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return fail(SERQ_ECUDA, "cuTensorMapEncodeTiled is unavailable");
+    const cuuint64_t dims[3] = {128, bytes / 512, 4};
+    const cuuint64_t strides[2] = {512, 128};
+    const cuuint32_t box[3] = {128, 2, 4};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(SERQ_ECUDA, "cuTensorMapEncodeTiled (scale view) failed (%d)", static_cast<int>(r));
+    return SERQ_OK;
 }
 
 serq_status make_map(CUtensorMap* map, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner,
@@ -897,9 +909,15 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
                                                                    static_cast<uint32_t*>(xsq),
                                                                    static_cast<float*>(xss));
     } else {
-        quant_act_mxfp4_kernel<<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint32_t*>(xq),
-                                                            static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
-                                                            static_cast<uint8_t*>(xss));
+        // flat stream over the M x K/8 chunks: up to 8 CTAs per SM, each warp
+        // taking 32 * QF_UNROLL chunks per pass
+        const long long chunks = static_cast<long long>(M) * (K / 8);
+        const long long per_cta = static_cast<long long>(kQuantThreads) * QF_UNROLL;
+        long long grid = (chunks + per_cta - 1) / per_cta;
+        if (grid > 8LL * info->sms) grid = 8LL * info->sms;
+        quant_act_mxfp4_flat_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, cs>>>(
+            X, M, K, r, rp, static_cast<uint32_t*>(xq), static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
+            static_cast<uint8_t*>(xss));
     }
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
@@ -1118,10 +1136,10 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.Y = static_cast<__nv_bfloat16*>(Y);
         const size_t row_blocks_a = static_cast<size_t>((M + 127) / 128);
         MxPairScaleMaps sf;
-        if (serq_status st = make_scale_map(&sf.sfa, xs, row_blocks_a * p.atoms_k_main * 512)) return st;
+        if (serq_status st = make_sfa_wide_map(&sf.sfa, xs, row_blocks_a * p.atoms_k_main * 512)) return st;
         sf.sfb = w->tm_wsf;
         if (rp > 0) {
-            if (serq_status st = make_scale_map(&sf.sfa_r, xss, row_blocks_a * p.atoms_k_res * 512)) return st;
+            if (serq_status st = make_sfa_wide_map(&sf.sfa_r, xss, row_blocks_a * p.atoms_k_res * 512)) return st;
         } else {
             sf.sfa_r = sf.sfa;
         }

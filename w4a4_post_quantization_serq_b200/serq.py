@@ -59,8 +59,12 @@ class SerqWeight:
         self.rp = ((r + 63) // 64) * 64 if r > 0 else 0
 
     def __del__(self):
-        if getattr(self, "handle", None) is not None and self.handle.value:
-            N.load().serq_weight_destroy(self.handle)
+        h = getattr(self, "handle", None)
+        if h is not None and h.value:
+            try:
+                N.load().serq_weight_destroy(h)
+            except Exception:  # interpreter shutdown: the library may already be gone
+                pass
             self.handle = None
 
     def view(self) -> Dict[str, torch.Tensor]:
