@@ -198,7 +198,8 @@ def quant_act_bytes(M: int, K: int, r: int, fmt: str) -> int:
     packed codes of X^_q and X~_{s,q} and their scales."""
     rp = ((r + 63) // 64) * 64 if r > 0 else 0
     scales = (M * K // 32 + M * rp // 32) if fmt == "mxfp4" else (4 * M + (4 * M if rp else 0))
-    return 2 * M * K + M * K // 2 + M * rp // 2 + scales
+    codes = (M * K + M * rp) if fmt == "w4a8" else (M * K // 2 + M * rp // 2)  # W4A8: one byte per code
+    return 2 * M * K + codes + scales
 
 
 def quant_roofline(layers, quant_ms, hbm_gbs):
@@ -619,6 +620,18 @@ def main():
                               "peak_source": "measured bf16 burst x 2 (nominal dense INT8/BF16 ratio); of measured",
                               "quant_act": quant_roofline(layers2, q2, peaks["hbm_gbs"])}
         del layers2
+        # W4A8: the same q_proj shape with INT8 activations (the abstract's second setting)
+        import dataclasses
+        wl8 = workload("qproj_int4")
+        wl8.linears = [dataclasses.replace(l, fmt="w4a8") for l in wl8.linears]
+        layers8 = build_layers(wl8)
+        t8, g8, q8 = time_steps(layers8, args.steps, args.warmup, None)
+        f8 = sum(L["flops"] for L in layers8)
+        line["w4a8_qproj"] = {"TOPS": f8 / (t8 / args.steps * 1e-3) / 1e12, "ms_per_step": t8 / args.steps,
+                              "serq_linear_us": g8[0] * 1e3,
+                              "frac_of_int8_peak": f8 / (g8[0] * 1e-3) / 1e12 / (peaks["bf16_tflops"] * 2),
+                              "quant_act": quant_roofline(layers8, q8, peaks["hbm_gbs"])}
+        del layers8
     if not args.no_extras and rank == 0:
         dec = bench_decode()
         line["decode"] = dec

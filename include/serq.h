@@ -23,6 +23,11 @@
  *                    activations, per output channel for W^ and R.
  *   SERQ_FMT_MXFP4 : E2M1 codes with one E8M0 exponent per 32 consecutive
  *                    elements along the reduction axis (OCP MX v1.0).
+ *   SERQ_FMT_W4A8  : the W4A8 setting of the arXiv abstract (fugumt.com): the
+ *                    weight side exactly as SERQ_FMT_INT4 (W^_q and Q(R) INT4
+ *                    per output channel); activations and the salient slice
+ *                    INT8 per token, s = max|x| / 127 (n = 8 in "基础量化"),
+ *                    codes in [-127, 127], one byte each (not packed).
  *
  * Conventions
  *   - Matrices are row-major. W is K x N (input channels x output channels,
@@ -66,7 +71,7 @@ typedef enum {
     SERQ_ETIMEOUT = 5      /* a kernel gave up waiting on a pipeline barrier */
 } serq_status;
 
-typedef enum { SERQ_FMT_INT4 = 0, SERQ_FMT_MXFP4 = 1 } serq_format;
+typedef enum { SERQ_FMT_INT4 = 0, SERQ_FMT_MXFP4 = 1, SERQ_FMT_W4A8 = 2 } serq_format;
 
 typedef struct serq_weight serq_weight; /* opaque prepared linear */
 
@@ -223,6 +228,8 @@ serq_status serq_fold_producer(const serq_weight* w, const void* src, int rows, 
  * serq_act_buffer_sizes):
  *   INT4 : xq u8[M][K/2], xs fp32[M] (= max_i|x|/7), xsq u8[M][rp/2], xss fp32[M]
  *          (= max_{i<r}|x|/7); codes rne(x / s) clipped to [-7, 7].
+ *   W4A8 : xq s8[M][K], xs fp32[M] (= max_i|x|/127), xsq s8[M][rp], xss fp32[M]
+ *          (= max_{i<r}|x|/127); codes rne(x / s) clipped to [-127, 127].
  *   MXFP4: xq u8[M][K/2], xs E8M0 atoms (M rows, K/32 blocks), xsq u8[M][rp/2],
  *          xss E8M0 atoms (M rows, rp/32 blocks; the slice's own blocks over
  *          its first r columns, a short last block padded with zeros).
@@ -270,17 +277,18 @@ serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, 
  * The SERQ linear (the "量化推理" formula): one kernel launch computing
  *   MXFP4: Y = bf16( sum over K of X^_q W^_q  +  sum over r of X~_{s,q} Q(R) ),
  *          both block-scaled products accumulated into one fp32 tile;
- *   INT4 : acc1 = sum_i qx qw, acc2 = sum_{i<r} qxs qR (int32, exact),
+ *   INT4, W4A8 : acc1 = sum_i qx qw, acc2 = sum_{i<r} qxs qR (int32, exact),
  *          Y = bf16(acc1 * xs[m] * w_scale[n] + acc2 * xss[m] * r_scale[n]).
  * Inputs are serq_quant_act's outputs for the same (M, K, r, fmt).
- * Y: device bf16 [M][N]. acc_dbg: NULL, or (INT4 only) device int32
+ * Y: device bf16 [M][N]. acc_dbg: NULL, or (INT4 weights: INT4, W4A8) device int32
  * [2][M][N] receiving acc1 and acc2.
  * Kernels (MXFP4): M <= 16 a split-K weight-streaming kernel (its split CTAs
  * form a thread-block cluster; launched with programmatic dependent launch,
  * so it may start streaming weights while the preceding kernel of the stream
  * finishes, and reads xq/xs and writes Y only after it completes);
  * 16 < M <= 128 a one-CTA tensor-core kernel; M > 128 a CTA-pair kernel.
- * INT4: one tensor-core kernel for every M. Results do not depend on which
+ * INT4 and W4A8: one tensor-core kernel for every M (W4A8 loads the int8
+ * activations straight into the MMA layout). Results do not depend on which
  * kernel ran beyond fp32 summation order (MXFP4); INT4 accumulators are exact.
  * Errors: EINVAL (shape/format mismatch with w, NULL/unaligned pointers),
  * EUNSUPPORTED (not an sm_100 device).

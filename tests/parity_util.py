@@ -45,7 +45,7 @@ def run_gpu(X: np.ndarray, W: np.ndarray, r: int, fmt: str, X_calib: np.ndarray 
     Xh = S.serq_fold_producer(w, Xd)
     qa = S.serq_quant_act(Xh, r, fmt)
     M, N = X.shape[0], W.shape[1]
-    acc = torch.zeros(2, M, N, dtype=torch.int32, device="cuda") if (acc_dbg and fmt == "int4") else None
+    acc = torch.zeros(2, M, N, dtype=torch.int32, device="cuda") if (acc_dbg and fmt in ("int4", "w4a8")) else None
     Y = S.serq_linear(w, qa, acc_dbg=acc)
     S.serq_device_status()
     view = w.view()
@@ -66,7 +66,7 @@ def expected_weight_bytes(prep: O.Prepared):
     r, rp = prep.r, rp_of(prep.r)
     N, K = prep.qw.shape
     out = {"perm": prep.perm, "s": prep.s, "inv_s": prep.inv_s, "wq": O.pack_nibbles(prep.qw)}
-    if prep.fmt == "int4":
+    if prep.fmt in O.INT_WEIGHT_FORMATS:
         out["w_scale"] = prep.sw
         if r > 0:
             out["rq"] = O.pack_nibbles(pad_cols(prep.qR, rp))
@@ -88,7 +88,7 @@ def compare_weight(got: dict, prep: O.Prepared):
     assert np.array_equal(v["s"].view(np.uint32), exp["s"].view(np.uint32)), "s"
     assert np.array_equal(v["inv_s"].view(np.uint32), exp["inv_s"].view(np.uint32)), "inv_s"
     assert np.array_equal(v["wq"], exp["wq"]), f"wq mismatch at {np.argwhere(v['wq'] != exp['wq'])[:5]}"
-    if prep.fmt == "int4":
+    if prep.fmt in O.INT_WEIGHT_FORMATS:
         assert np.array_equal(v["w_scale"].view(np.uint32), exp["w_scale"].view(np.uint32)), "sw"
         if prep.r > 0:
             assert np.array_equal(v["rq"], exp["rq"]), f"rq mismatch at {np.argwhere(v['rq'] != exp['rq'])[:5]}"
@@ -102,6 +102,15 @@ def compare_weight(got: dict, prep: O.Prepared):
 
 def compare_act(res: dict, qa: O.QuantAct, M: int, K: int, r: int):
     rp = rp_of(r)
+    if qa.fmt == "w4a8":  # one int8 code per element, fp32 scales
+        xq = res["xq"][: M * K].reshape(M, K).view(np.int8)
+        assert np.array_equal(xq, qa.qx), f"xq mismatch at {np.argwhere(xq != qa.qx)[:5]}"
+        assert np.array_equal(res["xs"].view(np.float32)[:M].view(np.uint32), qa.sx.view(np.uint32)), "sx"
+        if r > 0:
+            xsq = res["xsq"][: M * rp].reshape(M, rp).view(np.int8)
+            assert np.array_equal(xsq, pad_cols(qa.qxs, rp)), "xsq"
+            assert np.array_equal(res["xss"].view(np.float32)[:M].view(np.uint32), qa.sxs.view(np.uint32)), "sxs"
+        return
     xq = res["xq"][: M * K // 2].reshape(M, K // 2)
     assert np.array_equal(xq, O.pack_nibbles(qa.qx)), f"xq mismatch at {np.argwhere(xq != O.pack_nibbles(qa.qx))[:5]}"
     if qa.fmt == "int4":
@@ -137,7 +146,7 @@ def oracle_host_parts(prep: O.Prepared) -> dict:
     N, K = prep.qw.shape
     parts = {"perm": prep.perm.astype(np.int32), "s": prep.s.astype(np.float32),
              "inv_s": prep.inv_s.astype(np.float32), "wq": O.pack_nibbles(prep.qw)}
-    if prep.fmt == "int4":
+    if prep.fmt in O.INT_WEIGHT_FORMATS:
         parts["w_scale"] = prep.sw.astype(np.float32)
         parts["r_scale"] = prep.sR.astype(np.float32) if r > 0 else np.zeros(N, np.float32)
         parts["rq"] = O.pack_nibbles(pad_cols(prep.qR, rp)) if r > 0 else np.zeros((N, 0), np.uint8)

@@ -131,3 +131,8 @@ def test_quant_act_bytes_closed_form():
     # INT4, LLaMA-2-7B q_proj: fp32 per-token scales for the row and the slice
     assert bench.quant_act_bytes(2048, 4096, 128, "int4") == 2 * 2048 * 4096 + 2048 * 2048 + 2048 * 64 + 8 * 2048
     assert bench.quant_act_bytes(16, 4096, 0, "int4") == 2 * 16 * 4096 + 16 * 2048 + 4 * 16
+
+
+def test_quant_act_bytes_w4a8():
+    import bench
+    assert bench.quant_act_bytes(2048, 4096, 128, "w4a8") == 2 * 2048 * 4096 + 2048 * 4096 + 2048 * 128 + 8 * 2048

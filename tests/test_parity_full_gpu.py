@@ -5,6 +5,8 @@ bit for bit; Y and the INT4 accumulators on a seeded sample of token rows,
 which the oracle computes row by row.
 """
 
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -36,7 +38,7 @@ def _full(lin, M, rows_sample):
     w = S.serq_prepare(to_dev_bf16(W), lin.r, lin.fmt, act_absmax=a)
     Xh = S.serq_fold_producer(w, Xd)
     qa = S.serq_quant_act(Xh, lin.r, lin.fmt)
-    acc = torch.zeros(2, M, lin.N, dtype=torch.int32, device="cuda") if lin.fmt == "int4" else None
+    acc = torch.zeros(2, M, lin.N, dtype=torch.int32, device="cuda") if lin.fmt in ("int4", "w4a8") else None
     Y = S.serq_linear(w, qa, acc_dbg=acc)
     S.serq_device_status()
     res = {k: (None if getattr(qa, k) is None else getattr(qa, k).cpu().numpy()) for k in ("xq", "xs", "xsq", "xss")}
@@ -56,7 +58,7 @@ def _full(lin, M, rows_sample):
                      None if qa_o.Ex is None else qa_o.Ex[rows], qa_o.qxs[rows],
                      None if qa_o.sxs is None else qa_o.sxs[rows], None if qa_o.Exs is None else qa_o.Exs[rows])
     out = O.linear(prep, sub)
-    if lin.fmt == "int4":
+    if lin.fmt in ("int4", "w4a8"):
         acc_np = acc.cpu().numpy()
         assert np.array_equal(acc_np[0][rows], out.acc1)
         assert np.array_equal(acc_np[1][rows], out.acc2)
@@ -66,6 +68,12 @@ def _full(lin, M, rows_sample):
 def test_qproj_int4_full():
     wl = workload("qproj_int4")
     _full(wl.linears[0], wl.M, SAMPLE_ROWS)
+
+
+def test_qproj_w4a8_full():
+    # the W4A8 setting on the same LLaMA-2-7B q_proj shape (INT8 activations)
+    wl = workload("qproj_int4")
+    _full(dataclasses.replace(wl.linears[0], fmt="w4a8"), wl.M, SAMPLE_ROWS)
 
 
 @pytest.mark.parametrize("name", ["gate_up", "down"])

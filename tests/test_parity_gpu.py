@@ -2,7 +2,7 @@
 
 Bit-exact: calibration absmax, SAF scales, permutation, 1/s, folded
 activations, packed codes and scales of W^_q, Q(R), X^_q, X~_{s,q}, and the
-INT4 int32 accumulators. Within 2e-3 (max abs error over the row, divided by
+int32 accumulators of the INT4-weight formats (W4A4 INT4 and W4A8). Within 2e-3 (max abs error over the row, divided by
 the row's L2 norm): the bf16 output Y.
 """
 
@@ -29,20 +29,20 @@ def _check(X, W, r, fmt, X_calib=None):
     qa = O.quant_act(Xh, r, fmt)
     compare_act(res, qa, M, K, r)
     out = O.linear(prep, qa)
-    if fmt == "int4":
+    if fmt in ("int4", "w4a8"):
         assert np.array_equal(res["acc"][0], out.acc1), "acc1"
         assert np.array_equal(res["acc"][1], out.acc2), "acc2"
     return compare_y(res["Y"], out.Y)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
 def test_tiny_workload(fmt):
     wl = workload("tiny_int4")
     lin = wl.linears[0]
     _check(lin.X(wl.M), lin.W(), lin.r, fmt)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
 @pytest.mark.parametrize("M,K,N,r", [
     (1, 256, 256, 16),        # a single token
     (77, 384, 384, 32),       # ragged M, K % 256 == 128 (half K-tile), N % 256 == 128 (half N-tile)
@@ -61,7 +61,7 @@ def test_shapes(fmt, M, K, N, r):
     _check(X, W, r, fmt)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
 def test_degenerate_rows(fmt):
     # a zero row, an all-equal row, a row with one huge outlier, exact ties
     M, K, N, r = 8, 256, 256, 16
@@ -76,7 +76,7 @@ def test_degenerate_rows(fmt):
     _check(X, W, r, fmt, X_calib=X)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
 def test_calibration_on_separate_draw(fmt):
     M, K, N, r = 16, 512, 256, 128
     X = activations(21, M, K, 5, "const", 50.0)

@@ -38,7 +38,8 @@ def _res(qa):
             "xss": None if qa.xss is None else qa.xss.cpu().numpy()}
 
 
-RMS_CASES = [("int4", 64, 256, 256, 16), ("mxfp4", 64, 256, 256, 16), ("int4", 77, 384, 256, 40),
+RMS_CASES = [("int4", 64, 256, 256, 16), ("mxfp4", 64, 256, 256, 16), ("w4a8", 64, 256, 256, 16),
+             ("w4a8", 65, 20480, 128, 40), ("int4", 77, 384, 256, 40),
              ("mxfp4", 77, 384, 256, 40), ("mxfp4", 5, 1024, 512, 0), ("int4", 33, 20480, 128, 128),
              ("mxfp4", 129, 4096, 256, 128)]
 
@@ -61,7 +62,8 @@ def test_rmsnorm_quant_act(fmt, M, K, N, r):
     compare_act(_res(qa2), O.quant_act(Xh, r, fmt), M, K, r)
 
 
-SWI_CASES = [("int4", 64, 256, 256, 16), ("mxfp4", 64, 256, 256, 16), ("mxfp4", 77, 384, 256, 40),
+SWI_CASES = [("int4", 64, 256, 256, 16), ("mxfp4", 64, 256, 256, 16), ("w4a8", 77, 384, 256, 40),
+             ("mxfp4", 77, 384, 256, 40),
              ("int4", 77, 384, 256, 40), ("mxfp4", 3, 1024, 512, 0), ("int4", 9, 20480, 128, 128)]
 
 
@@ -86,7 +88,7 @@ def test_swiglu_quant_act(fmt, M, F, N, r):
     _swiglu_check(fmt, M, F, N, r, 70 + M)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
 def test_producer_then_linear(fmt):
     # RMSNorm -> gate/up-shaped linear, SwiGLU -> down-shaped linear
     M, K, F, r = 130, 512, 768, 32

@@ -11,7 +11,7 @@ LIB_PATH = os.path.join(_HERE, "libserq.so")
 HEADER = os.path.join(os.path.dirname(_HERE), "include", "serq.h")
 
 SERQ_OK, SERQ_EINVAL, SERQ_EUNSUPPORTED, SERQ_ENOMEM, SERQ_ECUDA, SERQ_ETIMEOUT = range(6)
-FMT = {"int4": 0, "mxfp4": 1}
+FMT = {"int4": 0, "mxfp4": 1, "w4a8": 2}
 STATUS_NAMES = {0: "SERQ_OK", 1: "SERQ_EINVAL", 2: "SERQ_EUNSUPPORTED", 3: "SERQ_ENOMEM",
                 4: "SERQ_ECUDA", 5: "SERQ_ETIMEOUT"}
 

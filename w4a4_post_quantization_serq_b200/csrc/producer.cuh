@@ -139,8 +139,23 @@ struct ProducerParams {
     __nv_bfloat16* xhat;     // NULL or debug copy of X^ [M][K]
 };
 
+// Hand a row of X^ to the quantizer of the consumer's format (0 INT4, 1 MXFP4,
+// 2 W4A8's INT8 activations).
+template <int FMT, int MAXC, class Src>
+__device__ __forceinline__ void quant_row(const Src& src, int m, int K, const ProducerParams& p, float* red) {
+    if constexpr (FMT == 0)
+        quant_row_int4<MAXC>(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<float*>(p.xs),
+                             static_cast<uint32_t*>(p.xsq), static_cast<float*>(p.xss), red);
+    else if constexpr (FMT == 1)
+        quant_row_mxfp4(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<uint8_t*>(p.xs),
+                        static_cast<uint32_t*>(p.xsq), static_cast<uint8_t*>(p.xss));
+    else
+        quant_row_int8<MAXC>(src, m, K, p.r, p.rp, static_cast<uint8_t*>(p.xq), static_cast<float*>(p.xs),
+                             static_cast<uint8_t*>(p.xsq), static_cast<float*>(p.xss), red);
+}
+
 // One CTA per token row. kind 0: RMSNorm of H (M x K); kind 1: SwiGLU of Y (M x 2K).
-// fmt 0: INT4 (MAXC chunks per thread), 1: MXFP4.
+// fmt 0: INT4, 2: INT8 (MAXC chunks per thread), 1: MXFP4.
 template <int KIND, int FMT, int MAXC>
 __global__ void __launch_bounds__(kQuantThreads)
 producer_quant_kernel(const uint4* __restrict__ in, const ProducerParams p) {
@@ -158,22 +173,12 @@ producer_quant_kernel(const uint4* __restrict__ in, const ProducerParams p) {
         const float ms = __fdiv_rn(__double2float_rn(ss), static_cast<float>(K));
         const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
         const SrcRmsNorm src{reinterpret_cast<const __nv_bfloat16*>(row), p.perm, p.inv_s, p.gamma, rstd, xhat_row};
-        if constexpr (FMT == 0)
-            quant_row_int4<MAXC>(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<float*>(p.xs),
-                                 static_cast<uint32_t*>(p.xsq), static_cast<float*>(p.xss), red);
-        else
-            quant_row_mxfp4(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<uint8_t*>(p.xs),
-                            static_cast<uint32_t*>(p.xsq), static_cast<uint8_t*>(p.xss));
+        quant_row<FMT, MAXC>(src, m, K, p, red);
     } else {
         stage_row(in + static_cast<size_t>(m) * (K >> 2), K >> 2, row, false);
         __syncthreads();
         const SrcSwiGlu src{reinterpret_cast<const __nv_bfloat16*>(row), K, p.perm, p.inv_s, xhat_row};
-        if constexpr (FMT == 0)
-            quant_row_int4<MAXC>(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<float*>(p.xs),
-                                 static_cast<uint32_t*>(p.xsq), static_cast<float*>(p.xss), red);
-        else
-            quant_row_mxfp4(src, m, K, p.r, p.rp, static_cast<uint32_t*>(p.xq), static_cast<uint8_t*>(p.xs),
-                            static_cast<uint32_t*>(p.xsq), static_cast<uint8_t*>(p.xss));
+        quant_row<FMT, MAXC>(src, m, K, p, red);
     }
 }
 

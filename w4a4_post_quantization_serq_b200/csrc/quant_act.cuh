@@ -160,6 +160,73 @@ __device__ __forceinline__ void quant_row_int4(const Src& src, int m, int K, int
     }
 }
 
+// INT8 code of x under scale s (the W4A8 activations): clip(rne(x / s), -127, 127)
+// as a byte; 0 when s == 0.
+__device__ __forceinline__ uint32_t int8_code(float x, float s) {
+    if (!(s > 0.0f)) return 0u;
+    float q = rintf(__fdiv_rn(x, s));
+    q = fminf(fmaxf(q, -127.0f), 127.0f);
+    return static_cast<uint32_t>(static_cast<int>(q)) & 0xFFu;
+}
+
+// INT8 (W4A8 activations), one CTA per row: s = max|x| / 127, one byte per code;
+// the salient slice under the absmax of its r columns. Same structure as INT4.
+template <int MAXC, class Src>
+__device__ __forceinline__ void quant_row_int8(const Src& src, int m, int K, int r, int rp, uint8_t* __restrict__ xq,
+                                               float* __restrict__ xs, uint8_t* __restrict__ xsq,
+                                               float* __restrict__ xss, float* red) {
+    const int nchunk = K >> 3;
+    uint4 v[MAXC];
+    float amax = 0.0f, amax_s = 0.0f;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = threadIdx.x + j * kQuantThreads;
+        if (c < nchunk) {
+            v[j] = src.chunk(c);
+            float f[8];
+            bf16x8_to_f32(v[j], f);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const float a = fabsf(f[e]);
+                amax = fmaxf(amax, a);
+                if (c * 8 + e < r) amax_s = fmaxf(amax_s, a);
+            }
+        }
+    }
+    block_max2(amax, amax_s, red);
+    const float s = __fdiv_rn(amax, 127.0f);
+    const float ss = __fdiv_rn(amax_s, 127.0f);
+    if (threadIdx.x == 0) {
+        xs[m] = s;
+        if (rp > 0) xss[m] = ss;
+    }
+    const int nchunk_s = rp >> 3;
+#pragma unroll
+    for (int j = 0; j < MAXC; ++j) {
+        const int c = threadIdx.x + j * kQuantThreads;
+        if (c < nchunk) {
+            float f[8];
+            bf16x8_to_f32(v[j], f);
+            uint32_t w0 = 0, w1 = 0;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                w0 |= int8_code(f[e], s) << (8 * e);
+                w1 |= int8_code(f[4 + e], s) << (8 * e);
+            }
+            *reinterpret_cast<uint2*>(xq + static_cast<size_t>(m) * K + c * 8) = make_uint2(w0, w1);
+            if (c < nchunk_s) {
+                uint32_t s0 = 0, s1 = 0;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    if (c * 8 + e < r) s0 |= int8_code(f[e], ss) << (8 * e);
+                    if (c * 8 + 4 + e < r) s1 |= int8_code(f[4 + e], ss) << (8 * e);
+                }
+                *reinterpret_cast<uint2*>(xsq + static_cast<size_t>(m) * rp + c * 8) = make_uint2(s0, s1);
+            }
+        }
+    }
+}
+
 // MXFP4, one CTA per row; four consecutive threads share one 32-element block.
 template <class Src>
 __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, int r, int rp,
@@ -213,11 +280,26 @@ __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, in
     }
 }
 
+template <int MAXC>
+__global__ void __launch_bounds__(kQuantThreads)
+quant_act_int8_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint8_t* __restrict__ xq,
+                      float* __restrict__ xs, uint8_t* __restrict__ xsq, float* __restrict__ xss) {
+    __shared__ float red[64];
+    pdl_launch_dependents();
+    const int m = blockIdx.x;
+    const SrcBf16Row src{X + static_cast<size_t>(m) * (K >> 3)};
+    quant_row_int8<MAXC>(src, m, K, r, rp, xq, xs, xsq, xss, red);
+}
+
 // MXFP4 serq_quant_act as a flat stream over all of X^: an MX block (32
 // values, four 16-byte chunks) never needs more than its own row segment, so
 // the grid walks the M x K/8 chunks directly. Each warp covers QF_UNROLL groups
 // of 32 consecutive chunks per pass (the four chunks of a block in four
-// consecutive lanes), with all its loads issued before any is used.
+// consecutive lanes), with all its loads issued before any is used. A group
+// starts on a multiple of 16 chunks of its row (K/8 is a multiple of 16), so
+// it spans at most two rows: the row index comes from one warp-uniform
+// division per group. The salient slice (the first rp columns) is handled
+// only by groups that reach into it.
 constexpr int QF_UNROLL = 4;
 
 __global__ void __launch_bounds__(kQuantThreads)
@@ -225,55 +307,69 @@ quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int M, int K, int r, in
                             uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
                             uint8_t* __restrict__ xss_atoms) {
     pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
-    const int nchunk = K >> 3;                 // chunks per row (a multiple of 16)
-    const int nchunk_s = rp >> 3;
+    const uint32_t nchunk = static_cast<uint32_t>(K) >> 3;    // chunks per row (a multiple of 16)
+    const uint32_t nchunk_s = static_cast<uint32_t>(rp) >> 3;
     const int atoms_k = (K / 32 + 3) / 4;
     const int atoms_s = (rp / 32 + 3) / 4;
-    const long long total = static_cast<long long>(M) * nchunk;
-    const int lane = threadIdx.x & 31;
-    const long long warp_id = (static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-    const long long n_warps = (static_cast<long long>(gridDim.x) * blockDim.x) >> 5;
-    for (long long base = warp_id * (32 * QF_UNROLL); base < total; base += n_warps * (32 * QF_UNROLL)) {
+    const uint32_t total = static_cast<uint32_t>(M) * nchunk;  // < 2^31 (M * K / 8)
+    const uint32_t lane = threadIdx.x & 31;
+    const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
+    for (uint32_t base = warp_id * (32 * QF_UNROLL); base < total; base += n_warps * (32 * QF_UNROLL)) {
         uint4 v[QF_UNROLL];
 #pragma unroll
         for (int u = 0; u < QF_UNROLL; ++u) {
-            const long long c = base + u * 32 + lane;
+            const uint32_t c = base + u * 32 + lane;
             v[u] = c < total ? __ldcs(X + c) : make_uint4(0u, 0u, 0u, 0u);
         }
 #pragma unroll
         for (int u = 0; u < QF_UNROLL; ++u) {
-            const long long c = base + u * 32 + lane;
-            const bool valid = c < total;          // uniform over each group of four lanes
-            const int m = valid ? static_cast<int>(c / nchunk) : 0;
-            const int cc = valid ? static_cast<int>(c - static_cast<long long>(m) * nchunk) : 0;
+            const uint32_t g0 = base + u * 32;                      // first chunk of the group
+            if (g0 >= total) break;                                  // warp-uniform
+            const uint32_t m0 = g0 / nchunk;
+            const uint32_t cc0 = g0 - m0 * nchunk;
+            const uint32_t cl = cc0 + lane;
+            const bool next = cl >= nchunk;
+            const uint32_t m = m0 + (next ? 1u : 0u);
+            const uint32_t cc = next ? cl - nchunk : cl;
+            const bool valid = m < static_cast<uint32_t>(M);        // uniform over each block of four lanes
             float f[8];
             bf16x8_to_f32(v[u], f);
-            float a = 0.0f, as = 0.0f;
+            float a = 0.0f;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-                a = fmaxf(a, fabsf(f[e]));
-                if (cc * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
-            }
+            for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(f[e]));
             a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
             a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
-            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+            // the salient slice: its own block maximum over the first r columns
+            const bool in_slice = valid && cc < nchunk_s;
+            float as = 0.0f;
+            if (__any_sync(0xFFFFFFFFu, in_slice)) {
+                if (in_slice) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (static_cast<int>(cc) * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
+                }
+                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+            }
             if (!valid) continue;
-            const int blk = cc >> 2;
+            const int blk = static_cast<int>(cc) >> 2;
             const int E = mx_exponent(a);
             const float inv = mx_inv_scale(E);
             float g[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
-            xq[c] = e2m1x8(g);
-            if ((lane & 3) == 0) xs_atoms[sf_atom_offset(m, blk, atoms_k)] = static_cast<uint8_t>(E + 127);
-            if (cc < nchunk_s) {
+            xq[static_cast<size_t>(m) * nchunk + cc] = e2m1x8(g);
+            if ((lane & 3) == 0)
+                xs_atoms[sf_atom_offset(static_cast<int>(m), blk, atoms_k)] = static_cast<uint8_t>(E + 127);
+            if (in_slice) {
                 const int Es = mx_exponent(as);
                 const float invs = mx_inv_scale(Es);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) g[e] = (cc * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+                for (int e = 0; e < 8; ++e) g[e] = (static_cast<int>(cc) * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
                 xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
-                if ((lane & 3) == 0) xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
+                if ((lane & 3) == 0)
+                    xss_atoms[sf_atom_offset(static_cast<int>(m), blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
             }
         }
     }

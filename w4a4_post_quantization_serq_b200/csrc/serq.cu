@@ -59,6 +59,9 @@ int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
 int residual_width(int r) { return r > 0 ? round_up(r, 64) : 0; }
 
+// INT4 weights (per-output-channel fp32 scales): the W4A4 and W4A8 formats.
+bool int_weights(int fmt) { return fmt == SERQ_FMT_INT4 || fmt == SERQ_FMT_W4A8; }
+
 size_t atom_bytes(int rows, int blocks) {
     return static_cast<size_t>((rows + 127) / 128) * static_cast<size_t>((blocks + 3) / 4) * 512u;
 }
@@ -235,7 +238,7 @@ std::atomic<int> g_fail_allocs{0};
 serq_status check_weight_shape(int K, int N, int r, int fmt) {
     if (K < 128 || K % 128 != 0 || K > 32768 || N < 128 || N % 128 != 0 || r < 0 || r > K)
         return fail(SERQ_EINVAL, "bad shape K=%d N=%d r=%d (need K%%128==0, K<=32768, N%%128==0, 0<=r<=K)", K, N, r);
-    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4) return fail(SERQ_EINVAL, "unknown format %d", fmt);
+    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4 && fmt != SERQ_FMT_W4A8) return fail(SERQ_EINVAL, "unknown format %d", fmt);
     return SERQ_OK;
 }
 
@@ -254,7 +257,7 @@ serq_status weight_alloc(int K, int N, int r, int fmt, int dev, cudaStream_t cs,
     w->device = dev;
     w->wq_bytes = static_cast<size_t>(N) * (K / 2);
     w->rq_bytes = static_cast<size_t>(N) * (rp / 2);
-    if (fmt == SERQ_FMT_INT4) {
+    if (int_weights(fmt)) {
         w->wsc_bytes = static_cast<size_t>(N) * 4;
         w->rsc_bytes = static_cast<size_t>(N) * 4;
     } else {
@@ -401,11 +404,15 @@ serq_status serq_act_buffer_sizes(int M, int K, int r, int fmt, serq_act_sizes* 
     if (out == nullptr) return fail(SERQ_EINVAL, "out is NULL");
     if (M < 1 || K < 128 || K % 128 != 0 || r < 0 || r > K)
         return fail(SERQ_EINVAL, "bad shape M=%d K=%d r=%d (need M>=1, K%%128==0, 0<=r<=K)", M, K, r);
-    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4) return fail(SERQ_EINVAL, "unknown format %d", fmt);
+    if (fmt != SERQ_FMT_INT4 && fmt != SERQ_FMT_MXFP4 && fmt != SERQ_FMT_W4A8) return fail(SERQ_EINVAL, "unknown format %d", fmt);
     const int rp = residual_width(r);
     out->xq = static_cast<size_t>(M) * (K / 2);
     out->xsq = static_cast<size_t>(M) * (rp / 2);
-    if (fmt == SERQ_FMT_INT4) {
+    if (fmt == SERQ_FMT_W4A8) {  // one int8 code per element
+        out->xq = static_cast<size_t>(M) * K;
+        out->xsq = static_cast<size_t>(M) * rp;
+    }
+    if (int_weights(fmt)) {
         out->xs = static_cast<size_t>(M) * 4;
         out->xss = rp > 0 ? static_cast<size_t>(M) * 4 : 0;
     } else {
@@ -488,7 +495,7 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     // fold + quantize W^, then the residual of the first r rows
     const dim3 qblock(32, 8);
     const dim3 qgrid(N / 32, (K / 32 + 7) / 8);
-    if (fmt == SERQ_FMT_INT4) {
+    if (int_weights(fmt)) {
         const int rows = 128;
         weight_colamax_kernel<<<dim3(N / 256 + (N % 256 != 0), (K + rows - 1) / rows), 256, 0, cs>>>(W, w->s, K, N,
                                                                                                     rows, tmp_col);
@@ -562,7 +569,7 @@ serq_status check_host_weight(const serq_weight_host* h) {
     }
     const size_t wq_bytes = static_cast<size_t>(N) * (K / 2);
     const size_t rq_row = static_cast<size_t>(rp / 2);
-    if (fmt == SERQ_FMT_INT4) {
+    if (int_weights(fmt)) {
         for (size_t i = 0; i < wq_bytes; ++i)
             if (!is_int4_code_ok(h->wq[i]) || !is_int4_code_ok(h->wq[i] >> 4))
                 return fail(SERQ_EINVAL, "INT4 code -8 in wq (byte %zu)", i);
@@ -596,7 +603,7 @@ serq_status check_host_weight(const serq_weight_host* h) {
             const uint8_t nib = (c & 1) ? (byte >> 4) : (byte & 0xF);
             if (nib != 0) return fail(SERQ_EINVAL, "rq row %d: nonzero code at position %d >= r", n, c);
         }
-    if (fmt == SERQ_FMT_INT4 && rp > 0)
+    if (int_weights(fmt) && rp > 0)
         for (size_t i = 0; i < static_cast<size_t>(N) * rq_row; ++i)
             if (!is_int4_code_ok(h->rq[i]) || !is_int4_code_ok(h->rq[i] >> 4))
                 return fail(SERQ_EINVAL, "INT4 code -8 in rq (byte %zu)", i);
@@ -761,7 +768,7 @@ serq_status serq_weight_export(const serq_weight* w, serq_weight_host* dst) {
         if (dst->wq != nullptr) SERQ_CUDA(cudaMemcpy(dst->wq, w->wq, w->wq_bytes, cudaMemcpyDeviceToHost));
         if (dst->rq != nullptr && w->rq_bytes > 0)
             SERQ_CUDA(cudaMemcpy(dst->rq, w->rq, w->rq_bytes, cudaMemcpyDeviceToHost));
-        if (w->fmt == SERQ_FMT_INT4) {
+        if (int_weights(w->fmt)) {
             if (dst->w_scale != nullptr) SERQ_CUDA(cudaMemcpy(dst->w_scale, w->wsc, 4u * N, cudaMemcpyDeviceToHost));
             if (dst->r_scale != nullptr) SERQ_CUDA(cudaMemcpy(dst->r_scale, w->rsc, 4u * N, cudaMemcpyDeviceToHost));
         } else {
@@ -812,7 +819,7 @@ serq_status serq_weight_create_from_host(const serq_weight_host* src, serq_weigh
     if (!st) st = up(w->wq, src->wq, w->wq_bytes);
     if (!st && rp > 0) st = up(w->rq, src->rq, w->rq_bytes);
     if (!st) {
-        if (src->fmt == SERQ_FMT_INT4) {
+        if (int_weights(src->fmt)) {
             st = up(w->wsc, src->w_scale, 4u * N);
             if (!st && src->r_scale != nullptr) st = up(w->rsc, src->r_scale, 4u * N);
         } else {
@@ -897,7 +904,16 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const int rp = residual_width(r);
     const uint4* X = static_cast<const uint4*>(Xhat);
-    if (fmt == SERQ_FMT_INT4) {
+    if (fmt == SERQ_FMT_W4A8) {
+        if (K <= 16384)
+            quant_act_int8_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint8_t*>(xq),
+                                                                  static_cast<float*>(xs), static_cast<uint8_t*>(xsq),
+                                                                  static_cast<float*>(xss));
+        else
+            quant_act_int8_kernel<16><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint8_t*>(xq),
+                                                                   static_cast<float*>(xs), static_cast<uint8_t*>(xsq),
+                                                                   static_cast<float*>(xss));
+    } else if (fmt == SERQ_FMT_INT4) {
         if (K <= 16384)
             quant_act_int4_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint32_t*>(xq),
                                                                   static_cast<float*>(xs),
@@ -910,8 +926,9 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
                                                                    static_cast<float*>(xss));
     } else {
         // flat stream over the M x K/8 chunks: up to 8 CTAs per SM, each warp
-        // taking 32 * QF_UNROLL chunks per pass
+        // taking 32 * QF_UNROLL chunks per pass (chunk indices are 32-bit)
         const long long chunks = static_cast<long long>(M) * (K / 8);
+        if (chunks >= (1LL << 31)) return fail(SERQ_EUNSUPPORTED, "M*K=%lld above 2^34", chunks * 8);
         const long long per_cta = static_cast<long long>(kQuantThreads) * QF_UNROLL;
         long long grid = (chunks + per_cta - 1) / per_cta;
         if (grid > 8LL * info->sms) grid = 8LL * info->sms;
@@ -939,9 +956,13 @@ serq_status producer_setup(DeviceInfo* info) {
     serq_status st = producer_setup_one<0, 0, 8>();
     if (!st) st = producer_setup_one<0, 0, 16>();
     if (!st) st = producer_setup_one<0, 1, 1>();
+    if (!st) st = producer_setup_one<0, 2, 8>();
+    if (!st) st = producer_setup_one<0, 2, 16>();
     if (!st) st = producer_setup_one<1, 0, 8>();
     if (!st) st = producer_setup_one<1, 0, 16>();
     if (!st) st = producer_setup_one<1, 1, 1>();
+    if (!st) st = producer_setup_one<1, 2, 8>();
+    if (!st) st = producer_setup_one<1, 2, 16>();
     if (!st) info->smem_set_prod = true;
     return st;
 }
@@ -980,21 +1001,23 @@ serq_status producer_launch(int kind, const serq_weight* w, const void* in, cons
     const uint4* src = static_cast<const uint4*>(in);
     const size_t smem = static_cast<size_t>(w->K) * (kind == 0 ? 2 : 4);
     const bool wide = w->K > 16384;
-    if (kind == 0) {
-        if (w->fmt == SERQ_FMT_MXFP4)
-            producer_quant_kernel<0, 1, 1><<<M, kQuantThreads, smem, cs>>>(src, p);
-        else if (wide)
-            producer_quant_kernel<0, 0, 16><<<M, kQuantThreads, smem, cs>>>(src, p);
-        else
-            producer_quant_kernel<0, 0, 8><<<M, kQuantThreads, smem, cs>>>(src, p);
-    } else {
-        if (w->fmt == SERQ_FMT_MXFP4)
-            producer_quant_kernel<1, 1, 1><<<M, kQuantThreads, smem, cs>>>(src, p);
-        else if (wide)
-            producer_quant_kernel<1, 0, 16><<<M, kQuantThreads, smem, cs>>>(src, p);
-        else
-            producer_quant_kernel<1, 0, 8><<<M, kQuantThreads, smem, cs>>>(src, p);
-    }
+    const int f = w->fmt;
+#define SERQ_PRODUCER(KIND)                                                                        \
+    do {                                                                                           \
+        if (f == SERQ_FMT_MXFP4)                                                                   \
+            producer_quant_kernel<KIND, 1, 1><<<M, kQuantThreads, smem, cs>>>(src, p);            \
+        else if (f == SERQ_FMT_INT4)                                                               \
+            (wide ? producer_quant_kernel<KIND, 0, 16> : producer_quant_kernel<KIND, 0, 8>)        \
+                <<<M, kQuantThreads, smem, cs>>>(src, p);                                          \
+        else                                                                                       \
+            (wide ? producer_quant_kernel<KIND, 2, 16> : producer_quant_kernel<KIND, 2, 8>)        \
+                <<<M, kQuantThreads, smem, cs>>>(src, p);                                          \
+    } while (0)
+    if (kind == 0)
+        SERQ_PRODUCER(0);
+    else
+        SERQ_PRODUCER(1);
+#undef SERQ_PRODUCER
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
 }
@@ -1022,7 +1045,7 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
     if (!aligned16(xq) || !aligned16(xs) || !aligned16(Y) || (w->rp > 0 && (!aligned16(xsq) || !aligned16(xss))) ||
         !aligned16(acc_dbg))
         return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
-    if (acc_dbg != nullptr && w->fmt != SERQ_FMT_INT4) return fail(SERQ_EINVAL, "acc_dbg is INT4-only");
+    if (acc_dbg != nullptr && !int_weights(w->fmt)) return fail(SERQ_EINVAL, "acc_dbg needs INT4 weights");
     int dev;
     DeviceInfo* info;
     if (serq_status st = device_check(&dev, &info)) return st;
@@ -1080,14 +1103,24 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         return SERQ_OK;
     }
 
-    const uint32_t bi = box_inner_bytes(w->fmt);
-    const bool swz = w->fmt == SERQ_FMT_MXFP4;
     CUtensorMap tm_a, tm_ar;
-    if (serq_status st = make_map(&tm_a, xq, K / 2, M, bi, 128, swz)) return st;
-    if (rp > 0) {
-        if (serq_status st = make_map(&tm_ar, xsq, rp / 2, M, bi, 128, swz)) return st;
+    if (w->fmt == SERQ_FMT_W4A8) {
+        // int8 activations: 128-byte rows of a K-tile, swizzled straight into the MMA layout
+        if (serq_status st = make_map(&tm_a, xq, K, M, 128, 128, true)) return st;
+        if (rp > 0) {
+            if (serq_status st = make_map(&tm_ar, xsq, rp, M, 128, 128, true)) return st;
+        } else {
+            tm_ar = tm_a;
+        }
     } else {
-        tm_ar = tm_a;
+        const uint32_t bi = box_inner_bytes(w->fmt);
+        const bool swz = w->fmt == SERQ_FMT_MXFP4;
+        if (serq_status st = make_map(&tm_a, xq, K / 2, M, bi, 128, swz)) return st;
+        if (rp > 0) {
+            if (serq_status st = make_map(&tm_ar, xsq, rp / 2, M, bi, 128, swz)) return st;
+        } else {
+            tm_ar = tm_a;
+        }
     }
     const int num_m = (M + 127) / 128;
     const int num_n = (N + 255) / 256;
@@ -1173,8 +1206,10 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         serq_linear_mxfp4_kernel<<<grid, mx::THREADS, mx::SMEM_BYTES, cs>>>(tm_a, w->tm_w, tm_ar, w->tm_r, p);
     } else {
         if (!info->smem_set_i4) {
-            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           i4::SMEM_BYTES));
+            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_int4_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           i4::Plan<false>::SMEM_BYTES));
+            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_int4_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                           i4::Plan<true>::SMEM_BYTES));
             info->smem_set_i4 = true;
         }
         I4Params p;
@@ -1192,7 +1227,12 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
         p.sR = static_cast<const float*>(w->rsc);
         p.Y = static_cast<__nv_bfloat16*>(Y);
         p.acc_dbg = acc_dbg;
-        serq_linear_int4_kernel<<<grid, i4::THREADS, i4::SMEM_BYTES, cs>>>(tm_a, w->tm_w, tm_ar, w->tm_r, p);
+        if (w->fmt == SERQ_FMT_W4A8)
+            serq_linear_int4_kernel<true><<<grid, i4::THREADS, i4::Plan<true>::SMEM_BYTES, cs>>>(tm_a, w->tm_w, tm_ar,
+                                                                                               w->tm_r, p);
+        else
+            serq_linear_int4_kernel<false><<<grid, i4::THREADS, i4::Plan<false>::SMEM_BYTES, cs>>>(tm_a, w->tm_w, tm_ar,
+                                                                                                 w->tm_r, p);
     }
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;

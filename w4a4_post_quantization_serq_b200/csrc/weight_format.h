@@ -8,8 +8,8 @@
 // 1/s are merged into the weights ahead of time, so they cost nothing at run
 // time). A checkpoint stores exactly that artefact in its canonical host form:
 //   perm int32[K], s fp32[K], inv_s fp32[K], wq u8[N][K/2],
-//   w_scale (INT4 fp32[N]; MXFP4 E8M0 u8[N][K/32]), rq u8[N][rp/2],
-//   r_scale (INT4 fp32[N]; MXFP4 E8M0 u8[N][rp/32])
+//   w_scale (INT4 weights fp32[N]; MXFP4 E8M0 u8[N][K/32]), rq u8[N][rp/2],
+//   r_scale (INT4 weights fp32[N]; MXFP4 E8M0 u8[N][rp/32])
 // in that order after a 64-byte header. Multi-byte fields are little-endian
 // (the byte order of every host this library builds for).
 #pragma once
@@ -35,7 +35,7 @@ struct Header {            // the first 64 bytes of a checkpoint file
 };
 static_assert(sizeof(Header) == kHeaderBytes, "checkpoint header must be 64 bytes");
 
-// Byte sizes of the canonical parts (fmt 0 = INT4, 1 = MXFP4).
+// Byte sizes of the canonical parts (fmt 0 = INT4, 1 = MXFP4, 2 = W4A8: INT4 weights).
 struct Sizes {
     size_t perm, s, inv_s, wq, w_scale, rq, r_scale;
     size_t total() const { return perm + s + inv_s + wq + w_scale + rq + r_scale; }
@@ -48,7 +48,7 @@ inline Sizes canonical_sizes(int fmt, int K, int N, int rp) {
     z.inv_s = z.perm;
     z.wq = static_cast<size_t>(N) * (K / 2);
     z.rq = static_cast<size_t>(N) * (rp / 2);
-    if (fmt == 0) {
+    if (fmt != 1) {
         z.w_scale = 4u * static_cast<size_t>(N);
         z.r_scale = 4u * static_cast<size_t>(N);
     } else {

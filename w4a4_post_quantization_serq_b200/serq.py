@@ -101,7 +101,7 @@ def serq_weight_get_view(w: SerqWeight) -> Dict[str, torch.Tensor]:
         "inv_s": _view(v.inv_s, (v.K,), "<f4", w),
         "wq": _view(v.wq, (v.N, v.K // 2), "|u1", w),
     }
-    if v.fmt == 0:
+    if v.fmt != N.FMT["mxfp4"]:  # INT4 weights (W4A4, W4A8): fp32 per-channel scales
         out["w_scale"] = _view(v.w_scale, (v.N,), "<f4", w)
         if v.rp > 0:
             out["rq"] = _view(v.rq, (v.N, v.rp // 2), "|u1", w)
@@ -118,7 +118,7 @@ def _host_parts(K: int, N_: int, r: int, rp: int, fmt: int) -> Dict[str, np.ndar
     """Zeroed numpy buffers of the canonical host form (see serq_weight_host in serq.h)."""
     out = {"perm": np.zeros(K, np.int32), "s": np.zeros(K, np.float32), "inv_s": np.zeros(K, np.float32),
            "wq": np.zeros((N_, K // 2), np.uint8), "rq": np.zeros((N_, rp // 2), np.uint8)}
-    if fmt == 0:
+    if fmt != N.FMT["mxfp4"]:
         out["w_scale"] = np.zeros(N_, np.float32)
         out["r_scale"] = np.zeros(N_, np.float32)
     else:
