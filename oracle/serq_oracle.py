@@ -431,6 +431,48 @@ def serq_forward(X: np.ndarray, W: np.ndarray, r: int, fmt: str,
 
 
 # ---------------------------------------------------------------------------
+# Two-factor baseline (L2QER)  [notes, "L2QER 的双矩阵路径"; gist-zh 1; gist-pt 1]
+#     Y^ = X_q W_q + Q(X_q L_{1,q}) L_{2,q}
+# The error correction uses two low-rank factors, so the intermediate
+# T = X_q L_{1,q} has to be quantized on the fly before the second product.
+# Here both factors live in the same folded frame as W^ (L1's rows follow the
+# SAF scales and permutation of the activations it multiplies), T leaves its
+# product in bf16 (a linear's output), and Q is the activation quantizer of
+# the format (per token for INT4, per 32 for MXFP4). SERQ's point of
+# comparison: one more GEMM, one more quantization, a serial dependency.
+# ---------------------------------------------------------------------------
+
+def prepare_given_residual(W: np.ndarray, R_given: np.ndarray, fmt: str, act_absmax: Optional[np.ndarray] = None,
+                           s: Optional[np.ndarray] = None) -> Prepared:
+    """W^_q exactly as prepare(W, 0, fmt), with the residual slot holding Q(R_given)
+    (R_given: k x N, quantized as Q(R) is) instead of W~_s - Q(W~_s)."""
+    base = prepare(W, 0, fmt, act_absmax=act_absmax, s=s)
+    R = np.asarray(R_given, dtype=F32)
+    k = R.shape[0]
+    Rt = np.ascontiguousarray(R.T)                        # [N, k]
+    if fmt in INT_WEIGHT_FORMATS:
+        qR, sR = quantize_int4(Rt, axis=1)
+        return dataclasses.replace(base, r=k, R=R, qR=qR, sR=sR)
+    qR, ER = quantize_mxfp4_rows(Rt)
+    return dataclasses.replace(base, r=k, R=R, qR=qR, ER=ER)
+
+
+def l2qer_linear(main: Prepared, l1: Prepared, qa: QuantAct, T_bf16: Optional[np.ndarray] = None) -> LinearOut:
+    """Y = X_q W_q + Q(T) L_{2,q}, T = X_q L_{1,q} stored in bf16.
+
+    main: prepare_given_residual(W, L2, ...); l1: prepare(L1, 0, ..., s = main.s)
+    (L1 folded with the main weight's scales and permutation); qa: quant_act(X^, 0).
+    T_bf16 replaces the bf16 intermediate (to check the later steps exactly)."""
+    assert l1.r == 0 and qa.r == 0 and np.array_equal(l1.perm, main.perm)
+    k = main.r
+    T = bf16_rne(linear(l1, qa).Y.astype(F32)) if T_bf16 is None else np.asarray(T_bf16, dtype=F32)
+    assert T.shape[1] == k
+    qT = quant_act(T, k, main.fmt)                         # on-the-fly quantization of T
+    res = QuantAct(main.fmt, k, qa.qx, qa.sx, qa.Ex, qT.qxs, qT.sxs, qT.Exs)
+    return linear(main, res)
+
+
+# ---------------------------------------------------------------------------
 # Producers with the offline fold merged in  [notes, Stage 3 "行/列排列离线合并到
 # 权重中"; gist-zh 2.3]: the layer that emits this linear's input writes X^
 # (permuted, divided by s) directly, so the activation quantization can run in

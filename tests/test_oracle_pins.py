@@ -577,3 +577,79 @@ def test_w4a8_brute_force_and_more_accurate_than_w4a4():
         assert np.max(np.abs(Yb - out.Y)) <= 1e-12 * np.max(np.abs(Yb))
         errs[fmt] = np.linalg.norm(out.Y - ref)
     assert errs["w4a8"] < errs["int4"]
+
+
+# --------------------------------------------------------------------------
+# the two-factor baseline (L2QER): Y = X_q W_q + Q(X_q L_{1,q}) L_{2,q}
+# ("L2QER 的双矩阵路径"); SERQ's comparison point for the latency overhead
+# --------------------------------------------------------------------------
+
+def _l2qer_setup(fmt, K=128, N=48, k=32, seed=101):
+    X = activations(seed, 12, K, 3, "lognormal", 40.0)
+    W = weights(seed + 1, K, N)
+    L1 = weights(seed + 2, K, k, 0.05)
+    L2 = weights(seed + 3, k, N, 0.01)
+    main = O.prepare_given_residual(W, L2, fmt, act_absmax=O.calib_absmax(X))
+    l1 = O.prepare(L1, 0, fmt, s=main.s)
+    qa = O.quant_act(O.fold_activation(X, main.s, main.perm), 0, fmt)
+    return X, W, L1, L2, main, l1, qa
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4", "w4a8"])
+def test_l2qer_zero_second_factor_is_plain_w4a4(fmt):
+    X, W, L1, L2, main, l1, qa = _l2qer_setup(fmt)
+    main0 = O.prepare_given_residual(W, np.zeros_like(L2), fmt, act_absmax=O.calib_absmax(X))
+    plain = O.linear(O.prepare(W, 0, fmt, act_absmax=O.calib_absmax(X)), qa)
+    assert np.array_equal(O.l2qer_linear(main0, l1, qa).Y, plain.Y)
+    # the main weight is the r = 0 preparation bit for bit
+    p0 = O.prepare(W, 0, fmt, act_absmax=O.calib_absmax(X))
+    assert np.array_equal(main.qw, p0.qw) and np.array_equal(main.perm, p0.perm)
+
+
+@pytest.mark.parametrize("fmt", ["int4", "mxfp4"])
+def test_l2qer_brute_force(fmt):
+    # every operand dequantized; T = X_q L1_q by a plain float64 matmul, rounded
+    # to bf16, quantized per token (INT4) / per 32 (MXFP4); then both products
+    X, W, L1, L2, main, l1, qa = _l2qer_setup(fmt)
+    T = qa.deq_x() @ l1.deq_w().T                               # [M, k] in the folded frame
+    T16 = O.bf16_rne(T.astype(np.float32))
+    if fmt == "int4":
+        q, s_ = O.quantize_int4(T16, axis=1)
+        Tq = q.astype(np.float64) * s_.astype(np.float64)[:, None]
+        L2q = O.quantize_int4(np.ascontiguousarray(L2.T), axis=1)
+        L2d = L2q[0].astype(np.float64) * L2q[1].astype(np.float64)[:, None]
+    else:
+        c, E = O.quantize_mxfp4_rows(T16)
+        Tq = O.mxfp4_dequant(c, E)
+        c2, E2 = O.quantize_mxfp4_rows(np.ascontiguousarray(L2.T))
+        L2d = O.mxfp4_dequant(c2, E2)
+    Y = qa.deq_x() @ main.deq_w().T + Tq @ L2d.T
+    got = O.l2qer_linear(main, l1, qa).Y
+    assert np.max(np.abs(got - Y)) <= 1e-12 * np.max(np.abs(Y))
+    # L1 is folded like W: the same product in the original frame
+    Xd = X.astype(np.float64)
+    assert np.allclose((Xd / main.s[None, :])[:, main.perm] @ l1.W_hat.astype(np.float64),
+                       Xd @ L1.astype(np.float64), rtol=1e-5, atol=1e-6)
+
+
+def test_l2qer_with_svd_factors_reduces_error():
+    # factors from the truncated SVD of the folded weight's quantization error
+    wl = workload("tiny_int4")
+    lin = wl.linears[0]
+    X, W = lin.X(wl.M), lin.W()
+    a = O.calib_absmax(X)
+    p0 = O.prepare(W, 0, "int4", act_absmax=a)
+    E = p0.W_hat.astype(np.float64) - p0.deq_w().T                # [K, N], folded frame
+    U, sv, Vt = np.linalg.svd(E, full_matrices=False)
+    k = 16
+    L1f = U[:, :k] * sv[:k]                                       # folded frame [K, k]
+    L1 = np.zeros_like(L1f)
+    L1[p0.perm] = L1f / p0.s[p0.perm].astype(np.float64)[:, None]  # back to the original frame
+    L2 = Vt[:k]
+    main = O.prepare_given_residual(W, L2.astype(np.float32), "int4", act_absmax=a)
+    l1 = O.prepare(L1.astype(np.float32), 0, "int4", s=main.s)
+    qa = O.quant_act(O.fold_activation(X, main.s, main.perm), 0, "int4")
+    ref = X.astype(np.float64) @ W.astype(np.float64)
+    err0 = np.linalg.norm(O.linear(p0, qa).Y - ref)
+    err2 = np.linalg.norm(O.l2qer_linear(main, l1, qa).Y - ref)
+    assert err2 < err0
