@@ -425,6 +425,48 @@ def bench_stack(ranks=(0, 16, 128, 256), reps: int = 3):
     return out
 
 
+def bench_l2qer(wl, steps: int, warmup: int, k: int = 128):
+    """The two-factor baseline on the same workload: per linear, serq_quant_act
+    (r = 0) then serq_linear_l2qer (T = X_q L1_q, Q(T), X_q W_q + Q(T) L2_q).
+    Synthetic factors L1 (K x k), L2 (k x N): the timing does not depend on
+    their values. Returns ms per step."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import weights
+    layers = []
+    for i, lin in enumerate(wl.linears):
+        X = torch.from_numpy(lin.X(wl.M)).to(torch.bfloat16).cuda()
+        W = torch.from_numpy(lin.W()).to(torch.bfloat16).cuda()
+        L1 = torch.from_numpy(weights(900 + i, lin.K, k, 0.05)).to(torch.bfloat16).cuda()
+        L2 = torch.from_numpy(weights(950 + i, k, lin.N, 0.01)).to(torch.bfloat16).cuda()
+        a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(wl.M)).to(torch.bfloat16).cuda())
+        main = S.serq_prepare(W, k, lin.fmt, act_absmax=a, R=L2)
+        l1 = S.serq_prepare(L1, 0, lin.fmt, s=main.view()["s"])
+        Xh = S.serq_fold_producer(main, X)
+        del X, W, L1, L2
+        layers.append({"main": main, "l1": l1, "Xh": Xh, "fmt": lin.fmt,
+                       "qa": S.alloc_act(wl.M, lin.K, 0, lin.fmt),
+                       "scratch": {"T": torch.empty(wl.M, k, dtype=torch.bfloat16, device="cuda"),
+                                   "tq": S.alloc_act(wl.M, k, k, lin.fmt)},
+                       "Y": torch.empty(wl.M, lin.N, dtype=torch.bfloat16, device="cuda")})
+
+    def step():
+        for L in layers:
+            S.serq_quant_act(L["Xh"], 0, L["fmt"], out=L["qa"])
+            S.serq_linear_l2qer(L["main"], L["l1"], L["qa"], Y=L["Y"], scratch=L["scratch"])
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step()
+    end.record()
+    torch.cuda.synchronize()
+    S.serq_device_status()
+    return start.elapsed_time(end) / steps
+
+
 # ----------------------------------------------------------------- CPU oracle
 def cpu_oracle_prepare(wl, r_override=None):
     """The oracle's offline preparation of every linear (not timed)."""
@@ -608,6 +650,13 @@ def main():
         torch.cuda.empty_cache()
         line["overhead_vs_r0"] = {"ms_per_step_r0": t0 / args.steps, "step": ms_per_step / (t0 / args.steps) - 1,
                                   "serq_linear": sum(gemm_ms) / sum(g0) - 1}
+        # the two-factor baseline (L2QER) at the same rank: its overhead over plain W4A4 against SERQ's
+        t_l2 = bench_l2qer(wl, args.steps, args.warmup)
+        ms_r0 = t0 / args.steps
+        line["l2qer"] = {"ms_per_step": t_l2, "rank": 128,
+                         "overhead_ms": t_l2 - ms_r0, "serq_overhead_ms": ms_per_step - ms_r0,
+                         "overhead_ratio_l2qer_over_serq": (t_l2 - ms_r0) / max(ms_per_step - ms_r0, 1e-9),
+                         "note": "steps with serq_quant_act; L2QER = T = X_q L1_q (bf16), Q(T), X_q W_q + Q(T) L2_q"}
         # INT4: LLaMA-2-7B q_proj shape
         wl2 = workload("qproj_int4")
         layers2 = build_layers(wl2)

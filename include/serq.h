@@ -107,6 +107,9 @@ typedef struct {
     const void* W;            /* device bf16 [K][N] */
     const float* act_absmax;  /* device fp32 [K], or NULL when s is given */
     const float* s;           /* device fp32 [K], or NULL */
+    const void* R;            /* NULL (SERQ: R = W~_s - Q(W~_s)), or device bf16 [r][N]: a given
+                                 matrix quantized into the residual slot instead (the second
+                                 factor of the two-factor baseline, serq_linear_l2qer) */
 } serq_prepare_desc;
 
 serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_stream stream);
@@ -296,6 +299,24 @@ serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, 
 serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void* xs,
                         const void* xsq, const void* xss, void* Y, int32_t* acc_dbg,
                         serq_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The two-factor baseline SERQ is compared against (L2QER; reading notes
+ * "L2QER 的双矩阵路径", gist.science/pt 1):
+ *     Y = X_q W_q + Q(X_q L_{1,q}) L_{2,q}
+ * Three launches, in order on `stream`: T = serq_linear(l1, X_q) (bf16
+ * [M][k] in the caller's scratch T), serq_quant_act(T, r = k) into tq/ts/
+ * tsq/tss (sizes serq_act_buffer_sizes(M, k, k, fmt)), then
+ * serq_linear(main, X_q, Q(T)) with Q(T) as the residual operand.
+ *   main: serq_prepare of W with desc.R = L2 (k x N) and r = k;
+ *   l1  : serq_prepare of L1 (K x k) with r = 0 and desc.s = main's SAF scales
+ *         (so L1 is folded with main's permutation and 1/s);
+ *   xq/xs: serq_quant_act(X^, r = 0) for main's K and format.
+ * k must meet serq_quant_act's rules (k % 128 == 0). Errors: those of the
+ * three calls, EINVAL for mismatched weights.
+ * ------------------------------------------------------------------------ */
+serq_status serq_linear_l2qer(const serq_weight* main, const serq_weight* l1, int M, const void* xq, const void* xs,
+                              void* T, void* tq, void* ts, void* tsq, void* tss, void* Y, serq_stream stream);
 
 /* ------------------------------------------------------------------------
  * serq_linear_small_m_noalloc — the small-M (M <= 16) MXFP4 linear for

@@ -16,6 +16,7 @@ from .serq import (  # noqa: F401
     serq_device_status,
     serq_fold_producer,
     serq_linear,
+    serq_linear_l2qer,
     serq_linear_small_m_noalloc,
     serq_prepare,
     serq_quant_act,

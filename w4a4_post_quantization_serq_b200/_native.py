@@ -20,7 +20,7 @@ c_int, c_size_t, c_void_p, c_char_p = ctypes.c_int, ctypes.c_size_t, ctypes.c_vo
 
 class PrepareDesc(ctypes.Structure):
     _fields_ = [("K", c_int), ("N", c_int), ("r", c_int), ("fmt", c_int),
-                ("W", c_void_p), ("act_absmax", c_void_p), ("s", c_void_p)]
+                ("W", c_void_p), ("act_absmax", c_void_p), ("s", c_void_p), ("R", c_void_p)]
 
 
 class WeightView(ctypes.Structure):
@@ -57,6 +57,8 @@ _SIGNATURES = {
                                       c_void_p]),
     "serq_linear": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p]),
+    "serq_linear_l2qer": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                  c_void_p, c_void_p, c_void_p, c_void_p]),
     "serq_linear_small_m_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                             c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "serq_weight_export": (c_int, [c_void_p, ctypes.POINTER(WeightHost)]),

@@ -247,6 +247,58 @@ __global__ void residual_mxfp4_kernel(const __nv_bfloat16* __restrict__ W, const
     r_atoms[sf_atom_offset(n, b, (rp / 32 + 3) / 4)] = static_cast<uint8_t>(Er + 127);
 }
 
+// Residual slot holding a given matrix G (r x N, bf16, row-major) instead of
+// W~_s - Q(W~_s): the second factor of the two-factor baseline (L2QER's L2).
+// Quantized exactly as Q(R) is.
+//   INT4 : thread per output channel n: s[n] = fp32(max_i |G[i, n]| / 7), codes rne(G / s)
+__global__ void given_residual_int4_kernel(const __nv_bfloat16* __restrict__ G, int N, int r, int rp,
+                                           uint8_t* __restrict__ rq, float* __restrict__ sR) {
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n >= N) return;
+    float a = 0.0f;
+    for (int i = 0; i < r; ++i) a = fmaxf(a, fabsf(bf16_at(G, static_cast<size_t>(i) * N + n)));
+    const float srn = __fdiv_rn(a, 7.0f);
+    sR[n] = srn;
+    for (int b = 0; b < rp / 32; ++b) {
+        uint32_t w[4] = {0u, 0u, 0u, 0u};
+        for (int e = 0; e < 32; ++e) {
+            const int i = b * 32 + e;
+            if (i < r) w[e >> 3] |= int4_code(bf16_at(G, static_cast<size_t>(i) * N + n), srn) << (4 * (e & 7));
+        }
+        *reinterpret_cast<uint4*>(rq + static_cast<size_t>(n) * (rp / 2) + b * 16) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+//   MXFP4: thread (n, 32-row block b along r): E8M0 exponent of the block, E2M1 codes
+__global__ void given_residual_mxfp4_kernel(const __nv_bfloat16* __restrict__ G, int N, int r, int rp,
+                                            uint8_t* __restrict__ rq, uint8_t* __restrict__ r_atoms) {
+    const int n = blockIdx.x * 32 + threadIdx.x;
+    const int b = blockIdx.y * blockDim.y + threadIdx.y;
+    if (n >= N || b * 32 >= rp) return;
+    float v[32];
+    float a = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const int i = b * 32 + e;
+        v[e] = i < r ? bf16_at(G, static_cast<size_t>(i) * N + n) : 0.0f;
+        a = fmaxf(a, fabsf(v[e]));
+    }
+    const int E = mx_exponent(a);
+    const float inv = mx_inv_scale(E);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float g[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(v[q * 8 + e], inv);
+        w[q] = e2m1x8(g);
+    }
+    *reinterpret_cast<uint4*>(rq + static_cast<size_t>(n) * (rp / 2) + b * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    // blocks past the last real one stay zero (padding)
+    if (b * 32 < r) r_atoms[sf_atom_offset(n, b, (rp / 32 + 3) / 4)] = static_cast<uint8_t>(E + 127);
+}
+
 // dst[row][i] = bf16(src[row][perm[i]] / s[perm[i]])  (Stage 3 producer fold)
 __global__ void fold_producer_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K,
                                      const int* __restrict__ perm, const float* __restrict__ s_perm,

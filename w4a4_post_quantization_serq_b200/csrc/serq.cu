@@ -459,6 +459,8 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     if (desc->W == nullptr || !aligned16(desc->W)) return fail(SERQ_EINVAL, "W must be a 16-byte aligned pointer");
     if ((desc->act_absmax == nullptr) == (desc->s == nullptr))
         return fail(SERQ_EINVAL, "give exactly one of act_absmax and s");
+    if (desc->R != nullptr && (!aligned16(desc->R) || r < 1))
+        return fail(SERQ_EINVAL, "a given residual needs r >= 1 and a 16-byte aligned pointer");
     int dev;
     DeviceInfo* info;
     if (serq_status st = device_check(&dev, &info)) return st;
@@ -482,6 +484,7 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
     } while (0)
 
     const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(desc->W);
+    const __nv_bfloat16* G = static_cast<const __nv_bfloat16*>(desc->R);  // given residual, or NULL
     // Stage 1: SAF scales
     if (desc->act_absmax != nullptr) {
         row_absmax_kernel<<<(K + 7) / 8, 256, 0, cs>>>(W, K, N, tmp_b);
@@ -501,14 +504,19 @@ serq_status serq_prepare(const serq_prepare_desc* desc, serq_weight** out, serq_
                                                                                                     rows, tmp_col);
         weight_quant_int4_kernel<<<qgrid, qblock, 0, cs>>>(W, w->perm, w->s_perm, tmp_col, K, N, w->wq,
                                                            static_cast<float*>(w->wsc));
-        if (r > 0)
+        if (r > 0 && G != nullptr)
+            given_residual_int4_kernel<<<(N + 127) / 128, 128, 0, cs>>>(G, N, r, rp, w->rq, static_cast<float*>(w->rsc));
+        else if (r > 0)
             residual_int4_kernel<<<(N + 127) / 128, 128, 0, cs>>>(W, w->perm, w->s_perm,
                                                                   static_cast<const float*>(w->wsc), N, r, rp, w->rq,
                                                                   static_cast<float*>(w->rsc));
     } else {
         weight_quant_mxfp4_kernel<<<qgrid, qblock, 0, cs>>>(W, w->perm, w->s_perm, K, N, w->wq,
                                                             static_cast<uint8_t*>(w->wsc));
-        if (r > 0)
+        if (r > 0 && G != nullptr)
+            given_residual_mxfp4_kernel<<<dim3(N / 32, (rp / 32 + 7) / 8), qblock, 0, cs>>>(
+                G, N, r, rp, w->rq, static_cast<uint8_t*>(w->rsc));
+        else if (r > 0)
             residual_mxfp4_kernel<<<dim3(N / 32, (rp / 32 + 7) / 8), qblock, 0, cs>>>(
                 W, w->perm, w->s_perm, K, N, r, rp, w->rq, static_cast<uint8_t*>(w->rsc));
     }
@@ -1236,6 +1244,18 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
     }
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
+}
+
+serq_status serq_linear_l2qer(const serq_weight* main, const serq_weight* l1, int M, const void* xq, const void* xs,
+                              void* T, void* tq, void* ts, void* tsq, void* tss, void* Y, serq_stream stream) {
+    if (main == nullptr || l1 == nullptr || T == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    if (l1->r != 0 || l1->K != main->K || l1->N != main->r || l1->fmt != main->fmt)
+        return fail(SERQ_EINVAL, "l1 must be K x k with r = 0 and main's format, k = main's r (%d)", main->r);
+    // T = X_q L1_q (bf16), then Q(T) on the fly, then X_q W_q + Q(T) L2_q in one launch
+    if (serq_status st = serq_linear(l1, M, xq, xs, nullptr, nullptr, T, nullptr, stream)) return st;
+    const int k = main->r;
+    if (serq_status st = serq_quant_act(T, M, k, k, main->fmt, tq, ts, tsq, tss, stream)) return st;
+    return serq_linear(main, M, xq, xs, tsq, tss, Y, nullptr, stream);
 }
 
 serq_status serq_linear_small_m_noalloc(int M, int K, int N, int r, const void* wq, const void* w_scale,

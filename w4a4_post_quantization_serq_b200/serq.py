@@ -81,12 +81,15 @@ def serq_calib_absmax(X: torch.Tensor, out: Optional[torch.Tensor] = None, strea
 
 
 def serq_prepare(W: torch.Tensor, r: int, fmt, act_absmax: Optional[torch.Tensor] = None,
-                 s: Optional[torch.Tensor] = None, stream=None) -> SerqWeight:
-    """Offline preparation of one linear; W is bf16 K x N (Y = X W). Synchronizes."""
+                 s: Optional[torch.Tensor] = None, R: Optional[torch.Tensor] = None, stream=None) -> SerqWeight:
+    """Offline preparation of one linear; W is bf16 K x N (Y = X W). Synchronizes.
+
+    R (bf16 r x N, optional) fills the residual slot with a given matrix (the
+    second factor of the two-factor baseline) instead of W~_s - Q(W~_s)."""
     if W.dtype != torch.bfloat16:
         raise ValueError("W must be bfloat16")
     K, N_ = W.shape
-    desc = N.PrepareDesc(K, N_, r, _fmt(fmt), _ptr(W), _ptr(act_absmax), _ptr(s))
+    desc = N.PrepareDesc(K, N_, r, _fmt(fmt), _ptr(W), _ptr(act_absmax), _ptr(s), _ptr(R))
     h = ctypes.c_void_p()
     N.check(N.load().serq_prepare(ctypes.byref(desc), ctypes.byref(h), _stream(stream)))
     return SerqWeight(h.value, K, N_, r, _fmt(fmt))
@@ -273,6 +276,21 @@ def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
         Y = torch.empty(qa.M, w.N, dtype=torch.bfloat16, device=qa.xq.device)
     N.check(N.load().serq_linear(w.handle, qa.M, _ptr(qa.xq), _ptr(qa.xs), _ptr(qa.xsq), _ptr(qa.xss), _ptr(Y),
                                  _ptr(acc_dbg), _stream(stream)))
+    return Y
+
+
+def serq_linear_l2qer(main: SerqWeight, l1: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
+                      scratch: Optional[dict] = None, stream=None) -> torch.Tensor:
+    """Two-factor baseline Y = X_q W_q + Q(X_q L1_q) L2_q (three launches; see serq.h)."""
+    M, k = qa.M, main.r
+    if scratch is None:
+        scratch = {"T": torch.empty(M, k, dtype=torch.bfloat16, device=qa.xq.device),
+                   "tq": alloc_act(M, k, k, main.fmt, qa.xq.device)}
+    if Y is None:
+        Y = torch.empty(M, main.N, dtype=torch.bfloat16, device=qa.xq.device)
+    t = scratch["tq"]
+    N.check(N.load().serq_linear_l2qer(main.handle, l1.handle, M, _ptr(qa.xq), _ptr(qa.xs), _ptr(scratch["T"]),
+                                       _ptr(t.xq), _ptr(t.xs), _ptr(t.xsq), _ptr(t.xss), _ptr(Y), _stream(stream)))
     return Y
 
 
