@@ -277,6 +277,35 @@ serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, 
                                   void* xss, void* xhat, serq_stream stream);
 
 /* ------------------------------------------------------------------------
+ * The SwiGLU producer fused into the gate/up linear's epilogue (MXFP4 only).
+ *
+ * serq_prepare_swiglu: `gate_up` describes [W_gate | W_up] (K x 2F, bf16,
+ *   device; SAF scales and rank of the gate/up linear as in serq_prepare),
+ *   `down` is the prepared down linear (K = F) it feeds. The down linear's
+ *   input permutation is merged into the gate/up weight's output columns
+ *   (Stage 3: "行/列排列离线合并到权重中"): column block t of 256 holds the
+ *   gate then the up columns of down's permuted input positions 128 t ..
+ *   128 t + 127. The weight keeps a copy of down's 1/s[perm] (F floats).
+ *   Quantization per output channel is unaffected by the arrangement.
+ *   Synchronizes. Errors: EINVAL, EUNSUPPORTED (not MXFP4), ENOMEM, ECUDA.
+ * serq_linear_swiglu_quant: the gate/up linear for M > 128 (CTA-pair
+ *   kernel) whose epilogue, instead of writing Y, computes for each row m and
+ *   permuted down channel i
+ *       X^_d[m,i] = bf16(fp32(fp32(silu(g) * u) * inv_s_d[i])),
+ *       silu(g) = g / (1 + expf(-g)) in fp32, g, u the fp32 accumulators,
+ *   and writes serq_quant_act's MXFP4 outputs for X^_d with down's rank:
+ *   hq/hs/hsq/hss sized by serq_act_buffer_sizes(M, F, down r, MXFP4).
+ *   xhat: NULL, or bf16 [M][F] receiving X^_d. xq..xss are gate/up's input
+ *   (serq_quant_act of its X^). M <= 128 returns EUNSUPPORTED (use
+ *   serq_linear and serq_swiglu_quant_act with an unarranged gate/up).
+ * ------------------------------------------------------------------------ */
+serq_status serq_prepare_swiglu(const serq_prepare_desc* gate_up, const serq_weight* down, serq_weight** out,
+                                serq_stream stream);
+serq_status serq_linear_swiglu_quant(const serq_weight* w, int M, const void* xq, const void* xs, const void* xsq,
+                                     const void* xss, void* hq, void* hs, void* hsq, void* hss, void* xhat,
+                                     serq_stream stream);
+
+/* ------------------------------------------------------------------------
  * The SERQ linear (the "量化推理" formula): one kernel launch computing
  *   MXFP4: Y = bf16( sum over K of X^_q W^_q  +  sum over r of X~_{s,q} Q(R) ),
  *          both block-scaled products accumulated into one fp32 tile;

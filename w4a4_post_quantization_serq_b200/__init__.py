@@ -18,7 +18,9 @@ from .serq import (  # noqa: F401
     serq_linear,
     serq_linear_l2qer,
     serq_linear_small_m_noalloc,
+    serq_linear_swiglu_quant,
     serq_prepare,
+    serq_prepare_swiglu,
     serq_quant_act,
     serq_rmsnorm_quant_act,
     serq_swiglu_quant_act,

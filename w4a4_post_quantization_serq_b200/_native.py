@@ -57,6 +57,9 @@ _SIGNATURES = {
                                       c_void_p]),
     "serq_linear": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p]),
+    "serq_prepare_swiglu": (c_int, [ctypes.POINTER(PrepareDesc), c_void_p, ctypes.POINTER(c_void_p), c_void_p]),
+    "serq_linear_swiglu_quant": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                         c_void_p, c_void_p, c_void_p, c_void_p, c_void_p]),
     "serq_linear_l2qer": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                   c_void_p, c_void_p, c_void_p, c_void_p]),
     "serq_linear_small_m_noalloc": (c_int, [c_int, c_int, c_int, c_int, c_void_p, c_void_p, c_void_p, c_void_p,

@@ -86,7 +86,80 @@ struct MxPairParams {
     int k_tiles_main, k_tiles_res;
     int atoms_k_main, atoms_k_res;
     __nv_bfloat16* Y;
+    // SwiGLU epilogue (EPI = 1): tile n_blk's columns are the gate (first 128) and
+    // up (last 128) outputs of the down linear's permuted input positions
+    // [128 n_blk, +128); the epilogue writes down's quantized input instead of Y.
+    int F, r_d, rp_d;               // down's K, rank and padded rank
+    const float* inv_s_d;           // [F] 1 / s_down[perm_down[i]]
+    uint32_t* hq;                   // [M][F / 8] words of eight E2M1 codes
+    uint8_t* hs;                    // E8M0 atoms over (M rows, F / 32 blocks)
+    uint32_t* hsq;                  // [M][rp_d / 8] salient slice codes
+    uint8_t* hss;                   // E8M0 atoms over (M rows, rp_d / 32 blocks)
+    __nv_bfloat16* xhat;            // NULL, or [M][F] debug copy of down's X^
 };
+
+// SwiGLU epilogue of one 32-channel block of one row: X^ = bf16(silu(g) u / s)
+// for permuted channels i0 .. i0+31, then the MX block (and, inside the first
+// r_d channels, the salient slice's own block) written as down's input.
+__device__ __forceinline__ void swiglu_quant_block(const MxPairParams& p, int m, int i0, const uint32_t (&g)[32],
+                                                   const uint32_t (&u)[32]) {
+    float x[32];
+    float amax = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+        const float gv = __uint_as_float(g[e]);
+        const float uv = __uint_as_float(u[e]);
+        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+        const float v = __fmul_rn(__fmul_rn(silu, uv), __ldg(p.inv_s_d + i0 + e));
+        x[e] = __bfloat162float(__float2bfloat16_rn(v));  // the bf16 X^ a stored producer output holds
+        amax = fmaxf(amax, fabsf(x[e]));
+    }
+    const int atoms_f = (p.F / 32 + 3) / 4;
+    const int E = mx_exponent(amax);
+    const float inv = mx_inv_scale(E);
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float t[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) t[e] = __fmul_rn(x[8 * q + e], inv);
+        w[q] = e2m1x8(t);
+    }
+    const size_t row_words = static_cast<size_t>(p.F) / 8;
+    *reinterpret_cast<uint4*>(p.hq + static_cast<size_t>(m) * row_words + i0 / 8) = make_uint4(w[0], w[1], w[2], w[3]);
+    p.hs[sf_atom_offset(m, i0 / 32, atoms_f)] = static_cast<uint8_t>(E + 127);
+    if (i0 < p.rp_d) {
+        // the slice's own block: the same block when it lies inside [0, r_d), else
+        // its absmax over the channels below r_d (zeros past r_d)
+        uint32_t ws[4] = {w[0], w[1], w[2], w[3]};
+        int Es = E;
+        if (i0 + 32 > p.r_d) {
+            float as = 0.0f;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+                if (i0 + e < p.r_d) as = fmaxf(as, fabsf(x[e]));
+            Es = mx_exponent(as);
+            const float invs = mx_inv_scale(Es);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float t[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) t[e] = (i0 + 8 * q + e < p.r_d) ? __fmul_rn(x[8 * q + e], invs) : 0.0f;
+                ws[q] = e2m1x8(t);
+            }
+        }
+        *reinterpret_cast<uint4*>(p.hsq + static_cast<size_t>(m) * (p.rp_d / 8) + i0 / 8) =
+            make_uint4(ws[0], ws[1], ws[2], ws[3]);
+        p.hss[sf_atom_offset(m, i0 / 32, (p.rp_d / 32 + 3) / 4)] = static_cast<uint8_t>(Es + 127);
+    }
+    if (p.xhat != nullptr) {
+        uint4* d = reinterpret_cast<uint4*>(p.xhat + static_cast<size_t>(m) * p.F + i0);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            d[q] = make_uint4(pack_bf16x2(x[8 * q], x[8 * q + 1]), pack_bf16x2(x[8 * q + 2], x[8 * q + 3]),
+                              pack_bf16x2(x[8 * q + 4], x[8 * q + 5]), pack_bf16x2(x[8 * q + 6], x[8 * q + 7]));
+    }
+}
 
 // Scale tensor maps (reads past the end give zeros). Activation atoms as a
 // 3-D view (x: 128 bytes, atom: stride 512, piece: stride 128) with box
@@ -97,6 +170,7 @@ struct MxPairScaleMaps {
     CUtensorMap sfa, sfb, sfa_r, sfb_r;
 };
 
+template <int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(mxp::THREADS, 1)
 serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b,
                               const __grid_constant__ CUtensorMap tm_ar, const __grid_constant__ CUtensorMap tm_br,
@@ -278,6 +352,38 @@ serq_linear_mxfp4_pair_kernel(const __grid_constant__ CUtensorMap tm_a, const __
             // on a timeout the warp skips the tile's work but keeps the tile-share barriers in step
             const bool ok =
                 __all_sync(0xFFFFFFFFu, mbar_wait(&acc_full[b], static_cast<uint32_t>((it >> 1) & 1), 0x331u));
+            if constexpr (EPI == 1) {
+                // SwiGLU epilogue: warp (quad, half) owns rows quad*32.. of this CTA and the
+                // permuted down channels [64 half, +64) of the tile: two 32-channel blocks,
+                // each read as its gate and up columns. The block holding the columns both
+                // accumulators share goes first (buffer 0: half 1, block 1 = up columns
+                // 224..255; buffer 1: half 0, block 0 = gate columns 0..31).
+                if (ok) {
+                    tc_fence_after();
+                    const uint32_t base = b ? TMEM_ACC1 : TMEM_ACC0;
+                    const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16) + base;
+                    const int m = m_pair * 2 * BM + static_cast<int>(rank) * BM + quad * 32 + lane;
+                    const bool owns_ovl = (b == 0 && half == 1) || (b == 1 && half == 0);
+                    const int first = b == 0 ? 1 : 0;
+#pragma unroll 1
+                    for (int jj = 0; jj < 2; ++jj) {
+                        const int j = owns_ovl ? (jj == 0 ? first : 1 - first) : jj;
+                        const int ch0 = 64 * half + 32 * j;
+                        uint32_t g[32], u[32];
+                        tmem_ld_32x32b_x32(t_lane + static_cast<uint32_t>(ch0), g);
+                        tmem_ld_32x32b_x32(t_lane + 128u + static_cast<uint32_t>(ch0), u);
+                        tmem_ld_wait();
+                        if (owns_ovl && jj == 0) {
+                            tc_fence_before();
+                            mbar_arrive_cluster(ovl_empty, 0);
+                        }
+                        if (m < p.M) swiglu_quant_block(p, m, n_blk * 128 + ch0, g, u);
+                    }
+                    tc_fence_before();
+                    mbar_arrive_cluster(&acc_empty[b], 0);
+                }
+                continue;
+            }
             uint32_t packed[64];
             if (ok) {
                 tc_fence_after();

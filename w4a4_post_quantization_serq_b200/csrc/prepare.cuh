@@ -299,6 +299,25 @@ __global__ void given_residual_mxfp4_kernel(const __nv_bfloat16* __restrict__ G,
     if (b * 32 < r) r_atoms[sf_atom_offset(n, b, (rp / 32 + 3) / 4)] = static_cast<uint8_t>(E + 127);
 }
 
+// Output columns of a gate/up weight [W_gate | W_up] (K x 2F) arranged for the
+// SwiGLU epilogue of the down linear it feeds (Stage 3: the down linear's
+// input permutation merged into the producer's weight): column block t
+// (256 wide) holds the gate then the up columns of down's permuted input
+// positions 128 t .. 128 t + 127:
+//   Wp[k][256 t + c]       = W[k][perm_d[128 t + c]]
+//   Wp[k][256 t + 128 + c] = W[k][F + perm_d[128 t + c]]
+__global__ void swiglu_arrange_kernel(const __nv_bfloat16* __restrict__ W, int K, int F, const int* __restrict__ perm_d,
+                                      __nv_bfloat16* __restrict__ Wp) {
+    const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+    const size_t cols = 2 * static_cast<size_t>(F);
+    if (idx >= static_cast<size_t>(K) * cols) return;
+    const size_t k = idx / cols;
+    const int col = static_cast<int>(idx - k * cols);
+    const int t = col >> 8, c = col & 255;
+    const int src = c < 128 ? perm_d[128 * t + c] : F + perm_d[128 * t + c - 128];
+    Wp[idx] = W[k * cols + src];
+}
+
 // dst[row][i] = bf16(src[row][perm[i]] / s[perm[i]])  (Stage 3 producer fold)
 __global__ void fold_producer_kernel(const __nv_bfloat16* __restrict__ src, int rows, int K,
                                      const int* __restrict__ perm, const float* __restrict__ s_perm,

@@ -227,6 +227,10 @@ struct serq_weight {
     CUtensorMap tm_rsf;
     float* tmp_b;          // preparation scratch at the end of the arena
     unsigned int* tmp_col;
+    // gate/up weight with the SwiGLU producer of a down linear folded in
+    // (serq_prepare_swiglu): its own allocation of down's 1/s[perm], F floats
+    float* swiglu_inv_s;
+    int swiglu_F, swiglu_r, swiglu_rp;
 };
 
 namespace {
@@ -441,11 +445,12 @@ serq_status serq_calib_absmax(const void* X, int M, int K, float* absmax, serq_s
 
 void serq_weight_destroy(serq_weight* w) {
     if (w == nullptr) return;
-    if (w->arena != nullptr) {
+    if (w->arena != nullptr || w->swiglu_inv_s != nullptr) {
         int cur = -1;
         cudaGetDevice(&cur);
         if (cur != w->device) cudaSetDevice(w->device);
-        cudaFree(w->arena);
+        if (w->arena != nullptr) cudaFree(w->arena);
+        if (w->swiglu_inv_s != nullptr) cudaFree(w->swiglu_inv_s);
         if (cur != w->device && cur >= 0) cudaSetDevice(cur);
     }
     delete w;
@@ -1030,6 +1035,65 @@ serq_status producer_launch(int kind, const serq_weight* w, const void* in, cons
     return SERQ_OK;
 }
 
+// CTA-pair MXFP4 kernel (M > 128): tile set-up and launch; `p` carries the
+// epilogue's outputs (Y, or for EPI = 1 the SwiGLU outputs).
+template <int EPI>
+serq_status launch_pair(const serq_weight* w, DeviceInfo* info, int M, const CUtensorMap& tm_a, const CUtensorMap& tm_ar,
+                        const void* xs, const void* xss, MxPairParams p, cudaStream_t cs) {
+    const int K = w->K, N = w->N, rp = w->rp;
+    if (!info->smem_set_mxp) {
+        SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_pair_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       mxp::SMEM_BYTES));
+        SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_pair_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       mxp::SMEM_BYTES));
+        cudaLaunchConfig_t qc = {};
+        qc.gridDim = dim3(info->sms, 1, 1);
+        qc.blockDim = dim3(mxp::THREADS, 1, 1);
+        qc.dynamicSmemBytes = mxp::SMEM_BYTES;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        qc.attrs = &attr;
+        qc.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, serq_linear_mxfp4_pair_kernel<0>, &qc) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = info->sms / 2;
+        }
+        info->pair_clusters = n;
+        info->smem_set_mxp = true;
+    }
+    p.M = M;
+    p.N = N;
+    p.K = K;
+    p.rp = rp;
+    p.num_n_tiles = (N + mxp::BN - 1) / mxp::BN;
+    p.num_m_pairs = (M + 2 * mxp::BM - 1) / (2 * mxp::BM);
+    p.num_tiles = p.num_n_tiles * p.num_m_pairs;
+    p.k_tiles_main = (K + mxp::BK - 1) / mxp::BK;
+    p.k_tiles_res = (rp + mxp::BK - 1) / mxp::BK;
+    p.atoms_k_main = K / 128;
+    p.atoms_k_res = (rp + 127) / 128;
+    const size_t row_blocks_a = static_cast<size_t>((M + 127) / 128);
+    MxPairScaleMaps sf;
+    if (serq_status st = make_sfa_wide_map(&sf.sfa, xs, row_blocks_a * p.atoms_k_main * 512)) return st;
+    sf.sfb = w->tm_wsf;
+    if (rp > 0) {
+        if (serq_status st = make_sfa_wide_map(&sf.sfa_r, xss, row_blocks_a * p.atoms_k_res * 512)) return st;
+    } else {
+        sf.sfa_r = sf.sfa;
+    }
+    sf.sfb_r = w->tm_rsf;
+    const int pairs = info->pair_clusters;
+    const int grid2 = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
+    serq_linear_mxfp4_pair_kernel<EPI><<<grid2, mxp::THREADS, mxp::SMEM_BYTES, cs>>>(tm_a, w->tm_w128, tm_ar,
+                                                                                    w->tm_r128, sf, p);
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -1137,58 +1201,9 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
 
     if (w->fmt == SERQ_FMT_MXFP4 && M > 128) {
         // CTA-pair kernel: 256 x 256 tiles, B halves split across the pair
-        if (!info->smem_set_mxp) {
-            SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_pair_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                           mxp::SMEM_BYTES));
-            cudaLaunchConfig_t qc = {};
-            qc.gridDim = dim3(info->sms, 1, 1);
-            qc.blockDim = dim3(mxp::THREADS, 1, 1);
-            qc.dynamicSmemBytes = mxp::SMEM_BYTES;
-            cudaLaunchAttribute attr;
-            attr.id = cudaLaunchAttributeClusterDimension;
-            attr.val.clusterDim.x = 2;
-            attr.val.clusterDim.y = 1;
-            attr.val.clusterDim.z = 1;
-            qc.attrs = &attr;
-            qc.numAttrs = 1;
-            int n = 0;
-            if (cudaOccupancyMaxActiveClusters(&n, serq_linear_mxfp4_pair_kernel, &qc) != cudaSuccess || n < 1) {
-                cudaGetLastError();
-                n = info->sms / 2;
-            }
-            info->pair_clusters = n;
-            info->smem_set_mxp = true;
-        }
-        CUtensorMap tm_b128, tm_br128;
-        tm_b128 = w->tm_w128;
-        tm_br128 = w->tm_r128;
-        MxPairParams p;
-        p.M = M;
-        p.N = N;
-        p.K = K;
-        p.rp = rp;
-        p.num_n_tiles = (N + mxp::BN - 1) / mxp::BN;
-        p.num_m_pairs = (M + 2 * mxp::BM - 1) / (2 * mxp::BM);
-        p.num_tiles = p.num_n_tiles * p.num_m_pairs;
-        p.k_tiles_main = (K + mxp::BK - 1) / mxp::BK;
-        p.k_tiles_res = (rp + mxp::BK - 1) / mxp::BK;
-        p.atoms_k_main = K / 128;
-        p.atoms_k_res = (rp + 127) / 128;
+        MxPairParams p{};
         p.Y = static_cast<__nv_bfloat16*>(Y);
-        const size_t row_blocks_a = static_cast<size_t>((M + 127) / 128);
-        MxPairScaleMaps sf;
-        if (serq_status st = make_sfa_wide_map(&sf.sfa, xs, row_blocks_a * p.atoms_k_main * 512)) return st;
-        sf.sfb = w->tm_wsf;
-        if (rp > 0) {
-            if (serq_status st = make_sfa_wide_map(&sf.sfa_r, xss, row_blocks_a * p.atoms_k_res * 512)) return st;
-        } else {
-            sf.sfa_r = sf.sfa;
-        }
-        sf.sfb_r = w->tm_rsf;
-        const int pairs = info->pair_clusters;
-        const int grid2 = 2 * (p.num_tiles < pairs ? p.num_tiles : pairs);
-        serq_linear_mxfp4_pair_kernel<<<grid2, mxp::THREADS, mxp::SMEM_BYTES, cs>>>(tm_a, tm_b128, tm_ar, tm_br128,
-                                                                                    sf, p);
+        if (serq_status st = launch_pair<0>(w, info, M, tm_a, tm_ar, xs, xss, p, cs)) return st;
     } else if (w->fmt == SERQ_FMT_MXFP4) {
         if (!info->smem_set_mx) {
             SERQ_CUDA(cudaFuncSetAttribute(serq_linear_mxfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1244,6 +1259,100 @@ serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void*
     }
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
+}
+
+serq_status serq_prepare_swiglu(const serq_prepare_desc* gate_up, const serq_weight* down, serq_weight** out,
+                                serq_stream stream) {
+    if (gate_up == nullptr || down == nullptr || out == nullptr) return fail(SERQ_EINVAL, "NULL argument");
+    *out = nullptr;
+    if (gate_up->fmt != SERQ_FMT_MXFP4 || down->fmt != SERQ_FMT_MXFP4)
+        return fail(SERQ_EUNSUPPORTED, "the fused SwiGLU epilogue is MXFP4 only");
+    const int F = down->K;
+    if (gate_up->N != 2 * F) return fail(SERQ_EINVAL, "gate/up N=%d must be 2 x down's K=%d", gate_up->N, F);
+    if (gate_up->R != nullptr) return fail(SERQ_EINVAL, "a given residual is not supported here");
+    if (serq_status st = check_weight_shape(gate_up->K, gate_up->N, gate_up->r, gate_up->fmt)) return st;
+    if (gate_up->W == nullptr || !aligned16(gate_up->W)) return fail(SERQ_EINVAL, "W must be a 16-byte aligned pointer");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    if (dev != down->device) return fail(SERQ_EINVAL, "down lives on device %d, current device is %d", down->device, dev);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const size_t elems = static_cast<size_t>(gate_up->K) * gate_up->N;
+    void* wp = nullptr;
+    float* inv = nullptr;
+    int pending = g_fail_allocs.load();
+    while (pending > 0 && !g_fail_allocs.compare_exchange_weak(pending, pending - 1)) {
+    }
+    if (pending > 0) return fail(SERQ_ENOMEM, "device allocation failed (injected by the test hook)");
+    if (cudaMalloc(&wp, elems * 2) != cudaSuccess) {
+        cudaGetLastError();
+        return fail(SERQ_ENOMEM, "cudaMalloc(%zu) for the arranged gate/up weight failed", elems * 2);
+    }
+    if (cudaMalloc(reinterpret_cast<void**>(&inv), sizeof(float) * F) != cudaSuccess) {
+        cudaGetLastError();
+        cudaFree(wp);
+        return fail(SERQ_ENOMEM, "cudaMalloc of down's 1/s failed");
+    }
+    auto cleanup = [&](serq_status st) {
+        cudaStreamSynchronize(cs);
+        cudaFree(wp);
+        if (inv != nullptr) cudaFree(inv);
+        return st;
+    };
+    swiglu_arrange_kernel<<<static_cast<unsigned>((elems + 255) / 256), 256, 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(gate_up->W), gate_up->K, F, down->perm, static_cast<__nv_bfloat16*>(wp));
+    if (cudaError_t e = cudaGetLastError()) return cleanup(cuda_fail(e, "swiglu_arrange_kernel"));
+    if (cudaError_t e = cudaMemcpyAsync(inv, down->inv_s, sizeof(float) * F, cudaMemcpyDeviceToDevice, cs))
+        return cleanup(cuda_fail(e, "cudaMemcpyAsync(down 1/s)"));
+    serq_prepare_desc d = *gate_up;
+    d.W = wp;
+    serq_weight* w = nullptr;
+    if (serq_status st = serq_prepare(&d, &w, stream)) return cleanup(st);  // synchronizes
+    cudaFree(wp);
+    w->swiglu_inv_s = inv;
+    w->swiglu_F = F;
+    w->swiglu_r = down->r;
+    w->swiglu_rp = down->rp;
+    *out = w;
+    return SERQ_OK;
+}
+
+serq_status serq_linear_swiglu_quant(const serq_weight* w, int M, const void* xq, const void* xs, const void* xsq,
+                                     const void* xss, void* hq, void* hs, void* hsq, void* hss, void* xhat,
+                                     serq_stream stream) {
+    if (w == nullptr) return fail(SERQ_EINVAL, "weight is NULL");
+    if (w->swiglu_F == 0) return fail(SERQ_EINVAL, "the weight was not prepared by serq_prepare_swiglu");
+    if (M <= 128) return fail(SERQ_EUNSUPPORTED, "the fused SwiGLU epilogue needs M > 128 (M=%d)", M);
+    if (xq == nullptr || xs == nullptr || hq == nullptr || hs == nullptr) return fail(SERQ_EINVAL, "NULL pointer");
+    if (w->rp > 0 && (xsq == nullptr || xss == nullptr)) return fail(SERQ_EINVAL, "r > 0 needs xsq and xss");
+    if (w->swiglu_rp > 0 && (hsq == nullptr || hss == nullptr)) return fail(SERQ_EINVAL, "down's r > 0 needs hsq and hss");
+    if (!aligned16(xq) || !aligned16(xs) || !aligned16(hq) || !aligned16(hs) || !aligned16(xhat) ||
+        (w->rp > 0 && (!aligned16(xsq) || !aligned16(xss))) || (w->swiglu_rp > 0 && (!aligned16(hsq) || !aligned16(hss))))
+        return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    if (dev != w->device) return fail(SERQ_EINVAL, "weight lives on device %d, current device is %d", w->device, dev);
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const int K = w->K, rp = w->rp;
+    CUtensorMap tm_a, tm_ar;
+    if (serq_status st = make_map(&tm_a, xq, K / 2, M, 128, 128, true)) return st;
+    if (rp > 0) {
+        if (serq_status st = make_map(&tm_ar, xsq, rp / 2, M, 128, 128, true)) return st;
+    } else {
+        tm_ar = tm_a;
+    }
+    MxPairParams p{};
+    p.F = w->swiglu_F;
+    p.r_d = w->swiglu_r;
+    p.rp_d = w->swiglu_rp;
+    p.inv_s_d = w->swiglu_inv_s;
+    p.hq = static_cast<uint32_t*>(hq);
+    p.hs = static_cast<uint8_t*>(hs);
+    p.hsq = static_cast<uint32_t*>(hsq);
+    p.hss = static_cast<uint8_t*>(hss);
+    p.xhat = static_cast<__nv_bfloat16*>(xhat);
+    return launch_pair<1>(w, info, M, tm_a, tm_ar, xs, xss, p, cs);
 }
 
 serq_status serq_linear_l2qer(const serq_weight* main, const serq_weight* l1, int M, const void* xq, const void* xs,

@@ -279,6 +279,31 @@ def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
     return Y
 
 
+def serq_prepare_swiglu(W_gate_up: torch.Tensor, r: int, down: SerqWeight, act_absmax: Optional[torch.Tensor] = None,
+                        s: Optional[torch.Tensor] = None, stream=None) -> SerqWeight:
+    """The gate/up linear ([W_gate | W_up], bf16 K x 2F) with down's permutation folded into its output
+    columns, for serq_linear_swiglu_quant. Synchronizes."""
+    K, N_ = W_gate_up.shape
+    desc = N.PrepareDesc(K, N_, r, N.FMT["mxfp4"], _ptr(W_gate_up), _ptr(act_absmax), _ptr(s), None)
+    h = ctypes.c_void_p()
+    N.check(N.load().serq_prepare_swiglu(ctypes.byref(desc), down.handle, ctypes.byref(h), _stream(stream)))
+    w = SerqWeight(h.value, K, N_, r, N.FMT["mxfp4"])
+    w.down = down
+    return w
+
+
+def serq_linear_swiglu_quant(w: SerqWeight, qa: QuantAct, out: Optional[QuantAct] = None,
+                             xhat: Optional[torch.Tensor] = None, stream=None) -> QuantAct:
+    """gate/up linear whose epilogue writes down's quantized input (SiLU(gate) * up, folded 1/s)."""
+    F = w.N // 2
+    if out is None:
+        out = alloc_act(qa.M, F, w.down.r, "mxfp4", qa.xq.device)
+    N.check(N.load().serq_linear_swiglu_quant(w.handle, qa.M, _ptr(qa.xq), _ptr(qa.xs), _ptr(qa.xsq), _ptr(qa.xss),
+                                              _ptr(out.xq), _ptr(out.xs), _ptr(out.xsq), _ptr(out.xss), _ptr(xhat),
+                                              _stream(stream)))
+    return out
+
+
 def serq_linear_l2qer(main: SerqWeight, l1: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
                       scratch: Optional[dict] = None, stream=None) -> torch.Tensor:
     """Two-factor baseline Y = X_q W_q + Q(X_q L1_q) L2_q (three launches; see serq.h)."""
