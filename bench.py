@@ -425,6 +425,60 @@ def bench_stack(ranks=(0, 16, 128, 256), reps: int = 3):
     return out
 
 
+def bench_mlp_fused(wl, steps: int, warmup: int):
+    """The MLP block with the producers fused (MXFP4, M = 2048): per step
+    serq_rmsnorm_quant_act (RMSNorm -> gate/up input, quantized) ->
+    serq_linear_swiglu_quant (gate/up whose epilogue writes down's quantized
+    input) -> serq_linear (down). Same linear flops as the headline step.
+    Returns (ms per step, per-launch us)."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import norm_weight
+    gu, dn = wl.linears
+    dev = "cuda"
+    Wd = torch.from_numpy(dn.W()).to(torch.bfloat16).to(dev)
+    w_d = S.serq_prepare(Wd, dn.r, dn.fmt,
+                         act_absmax=S.serq_calib_absmax(torch.from_numpy(dn.X_calib(wl.M)).to(torch.bfloat16).to(dev)))
+    Wgu = torch.from_numpy(gu.W()).to(torch.bfloat16).to(dev)
+    w_gu = S.serq_prepare_swiglu(Wgu, gu.r, w_d, act_absmax=S.serq_calib_absmax(
+        torch.from_numpy(gu.X_calib(wl.M)).to(torch.bfloat16).to(dev)))
+    del Wd, Wgu
+    H = torch.from_numpy(gu.X(wl.M)).to(torch.bfloat16).to(dev)      # the residual stream entering the MLP
+    gamma = torch.from_numpy(norm_weight(77, gu.K)).to(torch.bfloat16).to(dev)
+    qa = S.alloc_act(wl.M, gu.K, gu.r, gu.fmt, dev)
+    h = S.alloc_act(wl.M, dn.K, dn.r, dn.fmt, dev)
+    Y = torch.empty(wl.M, dn.N, dtype=torch.bfloat16, device=dev)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+
+    def step(record=False):
+        if record:
+            ev[0].record()
+        S.serq_rmsnorm_quant_act(w_gu, H, gamma, 1e-5, out=qa)
+        if record:
+            ev[1].record()
+        S.serq_linear_swiglu_quant(w_gu, qa, out=h)
+        if record:
+            ev[2].record()
+        S.serq_linear(w_d, h, Y=Y)
+        if record:
+            ev[3].record()
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    parts = [0.0, 0.0, 0.0]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for _ in range(steps):
+        step(record=True)
+        # per-launch split from the last step's events (read after the loop)
+    end.record()
+    torch.cuda.synchronize()
+    S.serq_device_status()
+    parts = [ev[i].elapsed_time(ev[i + 1]) * 1e3 for i in range(3)]
+    return start.elapsed_time(end) / steps, {"rmsnorm_quant_act": round(parts[0], 2),
+                                             "gate_up_swiglu_quant": round(parts[1], 2), "down": round(parts[2], 2)}
+
+
 def bench_l2qer(wl, steps: int, warmup: int, k: int = 128):
     """The two-factor baseline on the same workload: per linear, serq_quant_act
     (r = 0) then serq_linear_l2qer (T = X_q L1_q, Q(T), X_q W_q + Q(T) L2_q).
@@ -650,6 +704,12 @@ def main():
         torch.cuda.empty_cache()
         line["overhead_vs_r0"] = {"ms_per_step_r0": t0 / args.steps, "step": ms_per_step / (t0 / args.steps) - 1,
                                   "serq_linear": sum(gemm_ms) / sum(g0) - 1}
+        # the MLP block with the producers fused (RMSNorm -> quant, SwiGLU -> quant in the gate/up epilogue)
+        t_f, parts_f = bench_mlp_fused(wl, args.steps, args.warmup)
+        line["mlp_fused"] = {"ms_per_step": t_f, "TOPS": step_flops / (t_f * 1e-3) / 1e12, "per_launch_us": parts_f,
+                             "vs_unfused_step": ms_per_step / t_f,
+                             "note": "serq_rmsnorm_quant_act -> serq_linear_swiglu_quant -> serq_linear(down); "
+                                     "the unfused step has no RMSNorm or SwiGLU kernel at all"}
         # the two-factor baseline (L2QER) at the same rank: its overhead over plain W4A4 against SERQ's
         t_l2 = bench_l2qer(wl, args.steps, args.warmup)
         ms_r0 = t0 / args.steps
