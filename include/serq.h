@@ -292,7 +292,9 @@ serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, 
  *   kernel) whose epilogue, instead of writing Y, computes for each row m and
  *   permuted down channel i
  *       X^_d[m,i] = bf16(fp32(fp32(silu(g) * u) * inv_s_d[i])),
- *       silu(g) = g / (1 + expf(-g)) in fp32, g, u the fp32 accumulators,
+ *       silu(g) = g / (1 + exp(-g)) with the fast fp32 exponential and
+ *       division (a few ulp; X^_d is rounded to bf16 right after), g, u the
+ *       fp32 accumulators,
  *   and writes serq_quant_act's MXFP4 outputs for X^_d with down's rank:
  *   hq/hs/hsq/hss sized by serq_act_buffer_sizes(M, F, down r, MXFP4).
  *   xhat: NULL, or bf16 [M][F] receiving X^_d. xq..xss are gate/up's input

@@ -109,7 +109,8 @@ __device__ __forceinline__ void swiglu_quant_block(const MxPairParams& p, int m,
     for (int e = 0; e < 32; ++e) {
         const float gv = __uint_as_float(g[e]);
         const float uv = __uint_as_float(u[e]);
-        const float silu = __fdiv_rn(gv, __fadd_rn(1.0f, expf(-gv)));
+        // fast exp and division: the result is rounded to bf16 (8 bits) right after
+        const float silu = __fdividef(gv, 1.0f + __expf(-gv));
         const float v = __fmul_rn(__fmul_rn(silu, uv), __ldg(p.inv_s_d + i0 + e));
         x[e] = __bfloat162float(__float2bfloat16_rn(v));  // the bf16 X^ a stored producer output holds
         amax = fmaxf(amax, fabsf(x[e]));
