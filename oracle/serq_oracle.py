@@ -544,6 +544,56 @@ def swiglu_folded(Ygu: np.ndarray, perm: np.ndarray, inv_s: np.ndarray) -> np.nd
 
 
 # ---------------------------------------------------------------------------
+# The block around the SERQ linears (context for the time-to-first-token the
+# pages report for a LLaMA-3-8B 2K prefill  [notes, GPU 性能分析]): rotary
+# position embedding and causal grouped-query attention, both in float64.
+# The pages do not restate these layers; they are written in their standard
+# LLaMA form (rotate-half RoPE, softmax(q k^T / sqrt(d)) v with a causal mask,
+# query head h reading key/value head h // (n_q / n_kv)).
+# ---------------------------------------------------------------------------
+
+def rope(x: np.ndarray, n_heads: int, head_dim: int, base: float, pos0: int = 0) -> np.ndarray:
+    """Rotate-half RoPE of a token-major [M, n_heads * head_dim] array (float64):
+    for pair i < d/2 of each head, angle = (pos0 + m) * base^(-2i/d),
+    (x_i, x_{i+d/2}) -> (x_i cos - x_{i+d/2} sin, x_{i+d/2} cos + x_i sin)."""
+    x = np.asarray(x, dtype=np.float64)
+    M = x.shape[0]
+    h = x.reshape(M, n_heads, head_dim)
+    half = head_dim // 2
+    inv_freq = np.power(float(base), -np.arange(0, head_dim, 2, dtype=np.float64) / head_dim)
+    ang = (pos0 + np.arange(M, dtype=np.float64))[:, None] * inv_freq[None, :]
+    c, sn = np.cos(ang)[:, None, :], np.sin(ang)[:, None, :]
+    x1, x2 = h[..., :half], h[..., half:]
+    out = np.concatenate([x1 * c - x2 * sn, x2 * c + x1 * sn], axis=-1)
+    return out.reshape(M, n_heads * head_dim)
+
+
+def causal_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray, n_q: int, n_kv: int,
+                     head_dim: int) -> np.ndarray:
+    """softmax(q k^T / sqrt(d) + causal mask) v per query head, float64.
+    q: [M, n_q*d], k, v: [M, n_kv*d] (token-major); returns [M, n_q*d]."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    M = q.shape[0]
+    group = n_q // n_kv
+    out = np.zeros((M, n_q * head_dim))
+    mask = np.triu(np.ones((M, M), dtype=bool), 1)
+    for h in range(n_q):
+        g = h // group
+        qh = q[:, h * head_dim:(h + 1) * head_dim]
+        kh = k[:, g * head_dim:(g + 1) * head_dim]
+        vh = v[:, g * head_dim:(g + 1) * head_dim]
+        S = qh @ kh.T / np.sqrt(head_dim)
+        S[mask] = -np.inf
+        S = S - S.max(axis=1, keepdims=True)
+        P = np.exp(S)
+        P = P / P.sum(axis=1, keepdims=True)
+        out[:, h * head_dim:(h + 1) * head_dim] = P @ vh
+    return out
+
+
+# ---------------------------------------------------------------------------
 # canonical packed byte layouts used for bit-exact comparisons
 # ---------------------------------------------------------------------------
 

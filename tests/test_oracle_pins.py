@@ -653,3 +653,56 @@ def test_l2qer_with_svd_factors_reduces_error():
     err0 = np.linalg.norm(O.linear(p0, qa).Y - ref)
     err2 = np.linalg.norm(O.l2qer_linear(main, l1, qa).Y - ref)
     assert err2 < err0
+
+
+# --------------------------------------------------------------------------
+# the block around the linears (RoPE, causal GQA attention): closed forms
+# --------------------------------------------------------------------------
+
+def test_rope_closed_forms():
+    rng = np.random.default_rng(41)
+    nh, d = 3, 8
+    x = rng.standard_normal((5, nh * d))
+    y = O.rope(x, nh, d, 10000.0)
+    assert np.array_equal(y[0], x[0])                        # position 0: no rotation
+    # each (i, i + d/2) pair keeps its length
+    xr, yr = x.reshape(5, nh, d), y.reshape(5, nh, d)
+    n0 = xr[..., :4] ** 2 + xr[..., 4:] ** 2
+    n1 = yr[..., :4] ** 2 + yr[..., 4:] ** 2
+    assert np.allclose(n0, n1, rtol=1e-13)
+    # pair 0 turns by exactly m radians (base^0 = 1): a complex multiplication
+    m = 3
+    z = (xr[m, :, 0] + 1j * xr[m, :, 4]) * np.exp(1j * m)
+    assert np.allclose(yr[m, :, 0], z.real) and np.allclose(yr[m, :, 4], z.imag)
+    # scores depend only on the relative position: shifting both by t changes nothing
+    q, k = rng.standard_normal((1, d)), rng.standard_normal((1, d))
+    def score(pq, pk, t):
+        a = O.rope(q, 1, d, 500000.0, pos0=pq + t)
+        b = O.rope(k, 1, d, 500000.0, pos0=pk + t)
+        return float(a[0] @ b[0])
+    assert abs(score(7, 2, 0) - score(7, 2, 100)) < 1e-9
+
+
+def test_causal_attention_closed_forms():
+    rng = np.random.default_rng(42)
+    M, d, nq, nkv = 6, 4, 4, 2
+    q = rng.standard_normal((M, nq * d))
+    k = rng.standard_normal((M, nkv * d))
+    v = rng.standard_normal((M, nkv * d))
+    o = O.causal_attention(q, k, v, nq, nkv, d)
+    # the first token sees only itself: its output is its own value row (of its kv head)
+    for h in range(nq):
+        g = h // 2
+        assert np.allclose(o[0, h * d:(h + 1) * d], v[0, g * d:(g + 1) * d], rtol=1e-14)
+    # zero queries: uniform weights over the visible prefix
+    o0 = O.causal_attention(np.zeros_like(q), k, v, nq, nkv, d)
+    for m in range(M):
+        assert np.allclose(o0[m, :d], v[:m + 1, :d].mean(axis=0), rtol=1e-13)
+    # query heads 0, 1 share kv head 0, heads 2, 3 share kv head 1
+    q2 = q.copy()
+    q2[:, d:2 * d] = q[:, :d]
+    o2 = O.causal_attention(q2, k, v, nq, nkv, d)
+    assert np.allclose(o2[:, :d], o2[:, d:2 * d])
+    # a row is a convex combination of the visible values: inside their range
+    vis_max = np.maximum.accumulate(v[:, :d], axis=0)
+    assert np.all(o[:, :d] <= vis_max + 1e-12)
