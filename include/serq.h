@@ -308,6 +308,40 @@ serq_status serq_linear_swiglu_quant(const serq_weight* w, int M, const void* xq
                                      serq_stream stream);
 
 /* ------------------------------------------------------------------------
+ * The plain fold fused with the quantization, for a producer that cannot
+ * fold the permutation and 1/s into itself (the attention output feeding the
+ * o projection): X^[m,i] = bf16(X[m, perm[i]] / s[perm[i]]) (serq_fold_producer's
+ * arithmetic), then serq_quant_act's outputs for X^, in one pass. X: bf16
+ * [M][w->K]. xhat: NULL or a bf16 [M][K] copy of X^. Errors as above.
+ * ------------------------------------------------------------------------ */
+serq_status serq_fold_quant_act(const serq_weight* w, const void* X, int M, void* xq, void* xs, void* xsq, void* xss,
+                                void* xhat, serq_stream stream);
+
+/* ------------------------------------------------------------------------
+ * The LLaMA block around the SERQ linears (for the 2K-prefill time to first
+ * token the reading notes report under "GPU 性能分析"); standard definitions,
+ * bf16 storage, fp32 arithmetic.
+ *
+ * serq_rope: in place, rotate-half rotary embedding of heads [0, n_heads) of a
+ *   token-major bf16 matrix x (row stride ld elements, head h at columns
+ *   [h*head_dim, +head_dim)): for pair i < head_dim/2 at position pos0 + m,
+ *   angle = (pos0 + m) * base^(-2i/head_dim),
+ *   (x_i, x_{i+d/2}) <- (x_i cos - x_{i+d/2} sin, x_{i+d/2} cos + x_i sin).
+ * serq_attention_prefill: causal grouped-query attention, head_dim 128:
+ *   O_h = softmax(Q_h K_g^T / sqrt(128) + mask(key > query)) V_g,
+ *   g = h / (n_q / n_kv); q [M][ldq] (heads at column h*128), k, v [M][ldkv],
+ *   o [M][ldo]; all bf16, 16-byte aligned, leading dimensions multiples of 8.
+ *   Warp-level bf16 tensor-core MMAs with fp32 accumulation and an online
+ *   softmax (the scores never reach memory).
+ * serq_add: out = bf16(a + b) elementwise over n bf16 values (n % 8 == 0).
+ * All asynchronous on `stream`. Errors: EINVAL, EUNSUPPORTED (head_dim), ECUDA.
+ * ------------------------------------------------------------------------ */
+serq_status serq_rope(void* x, int M, int ld, int n_heads, int head_dim, float base, int pos0, serq_stream stream);
+serq_status serq_attention_prefill(const void* q, int ldq, const void* k, const void* v, int ldkv, int M, int n_q,
+                                   int n_kv, int head_dim, void* o, int ldo, serq_stream stream);
+serq_status serq_add(const void* a, const void* b, void* out, size_t n, serq_stream stream);
+
+/* ------------------------------------------------------------------------
  * The SERQ linear (the "量化推理" formula): one kernel launch computing
  *   MXFP4: Y = bf16( sum over K of X^_q W^_q  +  sum over r of X~_{s,q} Q(R) ),
  *          both block-scaled products accumulated into one fp32 tile;

@@ -11,10 +11,13 @@ from .serq import (  # noqa: F401
     SerqWeight,
     alloc_act,
     serq_act_buffer_sizes,
+    serq_add,
+    serq_attention_prefill,
     serq_calib_absmax,
     serq_debug_fail_next_allocations,
     serq_device_status,
     serq_fold_producer,
+    serq_fold_quant_act,
     serq_linear,
     serq_linear_l2qer,
     serq_linear_small_m_noalloc,
@@ -22,6 +25,7 @@ from .serq import (  # noqa: F401
     serq_prepare,
     serq_prepare_swiglu,
     serq_quant_act,
+    serq_rope,
     serq_rmsnorm_quant_act,
     serq_swiglu_quant_act,
     serq_selftest_wait,

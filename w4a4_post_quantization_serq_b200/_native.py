@@ -55,6 +55,12 @@ _SIGNATURES = {
                                        c_void_p, c_void_p, c_void_p, c_void_p]),
     "serq_swiglu_quant_act": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                                       c_void_p]),
+    "serq_fold_quant_act": (c_int, [c_void_p, c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                    c_void_p]),
+    "serq_rope": (c_int, [c_void_p, c_int, c_int, c_int, c_int, ctypes.c_float, c_int, c_void_p]),
+    "serq_attention_prefill": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_int, c_int, c_int, c_int, c_int,
+                                       c_void_p, c_int, c_void_p]),
+    "serq_add": (c_int, [c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]),
     "serq_linear": (c_int, [c_void_p, c_int, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
                             c_void_p]),
     "serq_prepare_swiglu": (c_int, [ctypes.POINTER(PrepareDesc), c_void_p, ctypes.POINTER(c_void_p), c_void_p]),

@@ -126,10 +126,29 @@ struct SrcSwiGlu {
     }
 };
 
+// X^ chunk of the plain fold (serq_fold_producer's arithmetic) of a row staged
+// in shared memory: X^[m,i] = bf16(X[m, perm[i]] / s[perm[i]]).
+struct SrcFold {
+    const __nv_bfloat16* x;
+    const int* perm;
+    const float* s_perm;
+    uint4* xhat;
+    __device__ __forceinline__ uint4 chunk(int c) const {
+        const PermChunk pc(perm, s_perm, c);  // .inv holds s[perm[i]] here
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = __fdiv_rn(__bfloat162float(x[pc.j[e]]), pc.inv[e]);
+        const uint4 out = pack_bf16x8(v);
+        if (xhat != nullptr) xhat[c] = out;
+        return out;
+    }
+};
+
 struct ProducerParams {
     int K, r, rp;            // the consuming linear's input width, rank, padded rank
     const int* perm;         // [K] permuted position -> producer channel
     const float* inv_s;      // [K] 1 / s[perm[i]]
+    const float* s_perm;     // [K] s[perm[i]] (the plain fold divides by it)
     const __nv_bfloat16* gamma;  // RMSNorm weight [K] (original order)
     float eps;
     void* xq;
@@ -154,7 +173,8 @@ __device__ __forceinline__ void quant_row(const Src& src, int m, int K, const Pr
                              static_cast<uint8_t*>(p.xsq), static_cast<float*>(p.xss), red);
 }
 
-// One CTA per token row. kind 0: RMSNorm of H (M x K); kind 1: SwiGLU of Y (M x 2K).
+// One CTA per token row. kind 0: RMSNorm of H (M x K); kind 1: SwiGLU of Y (M x 2K);
+// kind 2: the plain fold of X (M x K) (a producer that cannot fold itself).
 // fmt 0: INT4, 2: INT8 (MAXC chunks per thread), 1: MXFP4.
 template <int KIND, int FMT, int MAXC>
 __global__ void __launch_bounds__(kQuantThreads)
@@ -173,6 +193,11 @@ producer_quant_kernel(const uint4* __restrict__ in, const ProducerParams p) {
         const float ms = __fdiv_rn(__double2float_rn(ss), static_cast<float>(K));
         const float rstd = __fdiv_rn(1.0f, __fsqrt_rn(__fadd_rn(ms, p.eps)));
         const SrcRmsNorm src{reinterpret_cast<const __nv_bfloat16*>(row), p.perm, p.inv_s, p.gamma, rstd, xhat_row};
+        quant_row<FMT, MAXC>(src, m, K, p, red);
+    } else if constexpr (KIND == 2) {
+        stage_row(in + static_cast<size_t>(m) * (K >> 3), K >> 3, row, false);
+        __syncthreads();
+        const SrcFold src{reinterpret_cast<const __nv_bfloat16*>(row), p.perm, p.s_perm, xhat_row};
         quant_row<FMT, MAXC>(src, m, K, p, red);
     } else {
         stage_row(in + static_cast<size_t>(m) * (K >> 2), K >> 2, row, false);

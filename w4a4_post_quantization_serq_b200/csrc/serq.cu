@@ -19,6 +19,7 @@
 #include "ptx.cuh"
 #include "quant_act.cuh"
 #include "producer.cuh"
+#include "block.cuh"
 #include "prepare.cuh"
 #include "gemm_mxfp4.cuh"
 #include "gemm_int4.cuh"
@@ -976,6 +977,11 @@ serq_status producer_setup(DeviceInfo* info) {
     if (!st) st = producer_setup_one<1, 1, 1>();
     if (!st) st = producer_setup_one<1, 2, 8>();
     if (!st) st = producer_setup_one<1, 2, 16>();
+    if (!st) st = producer_setup_one<2, 0, 8>();
+    if (!st) st = producer_setup_one<2, 0, 16>();
+    if (!st) st = producer_setup_one<2, 1, 1>();
+    if (!st) st = producer_setup_one<2, 2, 8>();
+    if (!st) st = producer_setup_one<2, 2, 16>();
     if (!st) info->smem_set_prod = true;
     return st;
 }
@@ -1004,6 +1010,7 @@ serq_status producer_launch(int kind, const serq_weight* w, const void* in, cons
     p.rp = w->rp;
     p.perm = w->perm;
     p.inv_s = w->inv_s;
+    p.s_perm = w->s_perm;
     p.gamma = static_cast<const __nv_bfloat16*>(gamma);
     p.eps = eps;
     p.xq = xq;
@@ -1012,7 +1019,7 @@ serq_status producer_launch(int kind, const serq_weight* w, const void* in, cons
     p.xss = xss;
     p.xhat = static_cast<__nv_bfloat16*>(xhat);
     const uint4* src = static_cast<const uint4*>(in);
-    const size_t smem = static_cast<size_t>(w->K) * (kind == 0 ? 2 : 4);
+    const size_t smem = static_cast<size_t>(w->K) * (kind == 1 ? 4 : 2);
     const bool wide = w->K > 16384;
     const int f = w->fmt;
 #define SERQ_PRODUCER(KIND)                                                                        \
@@ -1028,8 +1035,10 @@ serq_status producer_launch(int kind, const serq_weight* w, const void* in, cons
     } while (0)
     if (kind == 0)
         SERQ_PRODUCER(0);
-    else
+    else if (kind == 1)
         SERQ_PRODUCER(1);
+    else
+        SERQ_PRODUCER(2);
 #undef SERQ_PRODUCER
     SERQ_CUDA(cudaGetLastError());
     return SERQ_OK;
@@ -1106,6 +1115,66 @@ serq_status serq_rmsnorm_quant_act(const serq_weight* w, const void* H, const vo
 serq_status serq_swiglu_quant_act(const serq_weight* w, const void* Ygu, int M, void* xq, void* xs, void* xsq,
                                   void* xss, void* xhat, serq_stream stream) {
     return producer_launch(1, w, Ygu, nullptr, 0.0f, M, xq, xs, xsq, xss, xhat, stream);
+}
+
+serq_status serq_fold_quant_act(const serq_weight* w, const void* X, int M, void* xq, void* xs, void* xsq, void* xss,
+                                void* xhat, serq_stream stream) {
+    return producer_launch(2, w, X, nullptr, 0.0f, M, xq, xs, xsq, xss, xhat, stream);
+}
+
+serq_status serq_rope(void* x, int M, int ld, int n_heads, int head_dim, float base, int pos0, serq_stream stream) {
+    if (x == nullptr || !aligned16(x)) return fail(SERQ_EINVAL, "x must be a 16-byte aligned pointer");
+    if (M < 1 || n_heads < 1 || head_dim < 2 || head_dim % 2 != 0 || ld < n_heads * head_dim || !(base > 1.0f) ||
+        pos0 < 0)
+        return fail(SERQ_EINVAL, "bad RoPE arguments M=%d ld=%d heads=%d dim=%d", M, ld, n_heads, head_dim);
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const size_t n = static_cast<size_t>(M) * n_heads * (head_dim / 2);
+    rope_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, cs>>>(static_cast<__nv_bfloat16*>(x), M, ld, n_heads,
+                                                                        head_dim, log2f(base), pos0);
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
+serq_status serq_attention_prefill(const void* q, int ldq, const void* k, const void* v, int ldkv, int M, int n_q,
+                                   int n_kv, int head_dim, void* o, int ldo, serq_stream stream) {
+    if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return fail(SERQ_EINVAL, "NULL pointer");
+    if (head_dim != att::D) return fail(SERQ_EUNSUPPORTED, "head_dim %d (only %d)", head_dim, att::D);
+    if (M < 1 || n_q < 1 || n_kv < 1 || n_q % n_kv != 0) return fail(SERQ_EINVAL, "bad M / head counts");
+    if (ldq < n_q * head_dim || ldkv < n_kv * head_dim || ldo < n_q * head_dim || ldq % 8 || ldkv % 8 || ldo % 8)
+        return fail(SERQ_EINVAL, "leading dimensions must cover the heads and be multiples of 8");
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+        return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    SERQ_CUDA(cudaFuncSetAttribute(attention_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   att::SMEM_BYTES));
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
+    attention_prefill_kernel<<<dim3((M + att::BM - 1) / att::BM, n_q), att::THREADS, att::SMEM_BYTES, cs>>>(
+        static_cast<const __nv_bfloat16*>(q), ldq, static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), ldkv, M, n_q, n_kv, scale_log2, static_cast<__nv_bfloat16*>(o), ldo);
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
+}
+
+serq_status serq_add(const void* a, const void* b, void* out, size_t n, serq_stream stream) {
+    if (a == nullptr || b == nullptr || out == nullptr || n % 8 != 0)
+        return fail(SERQ_EINVAL, "NULL pointer or n not a multiple of 8");
+    if (!aligned16(a) || !aligned16(b) || !aligned16(out)) return fail(SERQ_EINVAL, "pointers must be 16-byte aligned");
+    int dev;
+    DeviceInfo* info;
+    if (serq_status st = device_check(&dev, &info)) return st;
+    cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+    const size_t n8 = n / 8;
+    if (n8 > 0)
+        add_bf16_kernel<<<static_cast<unsigned>((n8 + 255) / 256), 256, 0, cs>>>(
+            static_cast<const uint4*>(a), static_cast<const uint4*>(b), static_cast<uint4*>(out), n8);
+    SERQ_CUDA(cudaGetLastError());
+    return SERQ_OK;
 }
 
 serq_status serq_linear(const serq_weight* w, int M, const void* xq, const void* xs, const void* xsq,

@@ -269,6 +269,51 @@ def serq_swiglu_quant_act(w: SerqWeight, Ygu: torch.Tensor, out: Optional[QuantA
     return out
 
 
+def serq_fold_quant_act(w: SerqWeight, X: torch.Tensor, out: Optional[QuantAct] = None,
+                        xhat: Optional[torch.Tensor] = None, stream=None) -> QuantAct:
+    """serq_fold_producer's fold and serq_quant_act in one pass (X: bf16 M x K)."""
+    M = X.shape[0]
+    if out is None:
+        out = alloc_act(M, w.K, w.r, w.fmt, X.device)
+    N.check(N.load().serq_fold_quant_act(w.handle, _ptr(X), M, _ptr(out.xq), _ptr(out.xs), _ptr(out.xsq),
+                                         _ptr(out.xss), _ptr(xhat), _stream(stream)))
+    return out
+
+
+def _strided_ptr(t: torch.Tensor) -> int:
+    """Pointer of a 2-D CUDA tensor whose rows are contiguous (a column slice of a row-major matrix)."""
+    if not t.is_cuda or t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError("expected a 2-D CUDA tensor with contiguous rows")
+    return t.data_ptr()
+
+
+def serq_rope(x: torch.Tensor, n_heads: int, head_dim: int, base: float, pos0: int = 0, stream=None) -> torch.Tensor:
+    """In-place rotate-half RoPE on the first n_heads heads of x (bf16 [M, >= n_heads*head_dim], rows contiguous)."""
+    N.check(N.load().serq_rope(_strided_ptr(x), x.shape[0], x.stride(0), n_heads, head_dim, float(base), pos0,
+                               _stream(stream)))
+    return x
+
+
+def serq_attention_prefill(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, n_q: int, n_kv: int,
+                           out: Optional[torch.Tensor] = None, head_dim: int = 128, stream=None) -> torch.Tensor:
+    """Causal grouped-query attention (bf16; q, k, v may be column slices of one QKV matrix)."""
+    M = q.shape[0]
+    if out is None:
+        out = torch.empty(M, n_q * head_dim, dtype=torch.bfloat16, device=q.device)
+    N.check(N.load().serq_attention_prefill(_strided_ptr(q), q.stride(0), _strided_ptr(k), _strided_ptr(v), k.stride(0),
+                                            M, n_q, n_kv, head_dim, _strided_ptr(out), out.stride(0),
+                                            _stream(stream)))
+    return out
+
+
+def serq_add(a: torch.Tensor, b: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """out = bf16(a + b) elementwise."""
+    if out is None:
+        out = torch.empty_like(a)
+    N.check(N.load().serq_add(_ptr(a), _ptr(b), _ptr(out), a.numel(), _stream(stream)))
+    return out
+
+
 def serq_linear(w: SerqWeight, qa: QuantAct, Y: Optional[torch.Tensor] = None,
                 acc_dbg: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
     """Y = X^_q W^_q + X~_{s,q} Q(R), bf16 M x N, in one kernel launch."""
