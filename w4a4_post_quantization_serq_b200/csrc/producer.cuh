@@ -176,8 +176,12 @@ __device__ __forceinline__ void quant_row(const Src& src, int m, int K, const Pr
 // One CTA per token row. kind 0: RMSNorm of H (M x K); kind 1: SwiGLU of Y (M x 2K);
 // kind 2: the plain fold of X (M x K) (a producer that cannot fold itself).
 // fmt 0: INT4, 2: INT8 (MAXC chunks per thread), 1: MXFP4.
+// Several CTAs per SM: a row is a short job (one read of the row, its
+// quantization), so the SM needs several rows in flight to hide the latency.
+// MXFP4 rows hold nothing across the row (4 CTAs per SM); the per-token
+// integer formats keep the row's chunks in registers (MAXC of them).
 template <int KIND, int FMT, int MAXC>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, FMT == 1 ? 4 : (MAXC > 8 ? 2 : 3))
 producer_quant_kernel(const uint4* __restrict__ in, const ProducerParams p) {
     extern __shared__ __align__(16) uint8_t smem_prod[];
     __shared__ double red64[kQuantThreads / 32];

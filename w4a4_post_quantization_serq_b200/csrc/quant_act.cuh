@@ -291,86 +291,84 @@ quant_act_int8_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint8_t
     quant_row_int8<MAXC>(src, m, K, r, rp, xq, xs, xsq, xss, red);
 }
 
-// MXFP4 serq_quant_act as a flat stream over all of X^: an MX block (32
-// values, four 16-byte chunks) never needs more than its own row segment, so
-// the grid walks the M x K/8 chunks directly. Each warp covers QF_UNROLL groups
-// of 32 consecutive chunks per pass (the four chunks of a block in four
-// consecutive lanes), with all its loads issued before any is used. A group
-// starts on a multiple of 16 chunks of its row (K/8 is a multiple of 16), so
-// it spans at most two rows: the row index comes from one warp-uniform
-// division per group. The salient slice (the first rp columns) is handled
-// only by groups that reach into it.
+// MXFP4 serq_quant_act as a stream over X^: an MX block (32 values, four
+// 16-byte chunks) needs nothing beyond its own row segment, so no row-wide
+// reduction is needed. Grid (ceil(K/8 / QF_CHUNKS), M): a CTA owns one
+// segment of QF_CHUNKS chunks of one row, each warp QF_UNROLL groups of 32
+// consecutive chunks (the four chunks of a block in four consecutive lanes),
+// all of its loads issued before any is used. The row is blockIdx.y, so the
+// addressing is a few adds; the salient slice is handled only by groups that
+// reach into the first rp columns.
 constexpr int QF_UNROLL = 4;
+constexpr int QF_THREADS = 128;
+constexpr int QF_CHUNKS = QF_THREADS * QF_UNROLL;  // 512 chunks = 4096 values of a row per CTA
 
-__global__ void __launch_bounds__(kQuantThreads)
-quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int M, int K, int r, int rp, uint32_t* __restrict__ xq,
+__global__ void __launch_bounds__(QF_THREADS)
+quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
                             uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
                             uint8_t* __restrict__ xss_atoms) {
     pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
-    const uint32_t nchunk = static_cast<uint32_t>(K) >> 3;    // chunks per row (a multiple of 16)
-    const uint32_t nchunk_s = static_cast<uint32_t>(rp) >> 3;
+    const int nchunk = K >> 3;
+    const int nchunk_s = rp >> 3;
+    const int m = blockIdx.y;
+    const int lane = threadIdx.x & 31;
+    const int c_base = blockIdx.x * QF_CHUNKS + (threadIdx.x >> 5) * (32 * QF_UNROLL);
+    const uint4* row = X + static_cast<size_t>(m) * nchunk;
+    uint4 v[QF_UNROLL];
+#pragma unroll
+    for (int u = 0; u < QF_UNROLL; ++u) {
+        const int cc = c_base + u * 32 + lane;
+        v[u] = cc < nchunk ? __ldcs(row + cc) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    // this row's scale atoms: row part of the offset fixed, block part per lane
     const int atoms_k = (K / 32 + 3) / 4;
     const int atoms_s = (rp / 32 + 3) / 4;
-    const uint32_t total = static_cast<uint32_t>(M) * nchunk;  // < 2^31 (M * K / 8)
-    const uint32_t lane = threadIdx.x & 31;
-    const uint32_t warp_id = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const uint32_t n_warps = (gridDim.x * blockDim.x) >> 5;
-    for (uint32_t base = warp_id * (32 * QF_UNROLL); base < total; base += n_warps * (32 * QF_UNROLL)) {
-        uint4 v[QF_UNROLL];
+    const size_t row_sf = static_cast<size_t>(m & 31) * 16 + static_cast<size_t>((m >> 5) & 3) * 4;
+    uint8_t* xs_row = xs_atoms + static_cast<size_t>(m >> 7) * atoms_k * 512 + row_sf;
+    uint32_t* xq_row = xq + static_cast<size_t>(m) * nchunk;
 #pragma unroll
-        for (int u = 0; u < QF_UNROLL; ++u) {
-            const uint32_t c = base + u * 32 + lane;
-            v[u] = c < total ? __ldcs(X + c) : make_uint4(0u, 0u, 0u, 0u);
+    for (int u = 0; u < QF_UNROLL; ++u) {
+        const int g0 = c_base + u * 32;
+        if (g0 >= nchunk) break;                       // warp-uniform
+        const int cc = g0 + lane;
+        const bool valid = cc < nchunk;                // uniform over each block of four lanes
+        float f[8];
+        bf16x8_to_f32(v[u], f);
+        float a = 0.0f;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(f[e]));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+        // the salient slice: its own block maximum over the first r columns
+        const bool slice_group = g0 < nchunk_s;       // warp-uniform (nchunk_s is a multiple of 8)
+        float as = 0.0f;
+        if (slice_group) {
+            if (valid && cc < nchunk_s) {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (cc * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
+            }
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
         }
+        if (!valid) continue;
+        const int blk = cc >> 2;
+        const int E = mx_exponent(a);
+        const float inv = mx_inv_scale(E);
+        float g[8];
 #pragma unroll
-        for (int u = 0; u < QF_UNROLL; ++u) {
-            const uint32_t g0 = base + u * 32;                      // first chunk of the group
-            if (g0 >= total) break;                                  // warp-uniform
-            const uint32_t m0 = g0 / nchunk;
-            const uint32_t cc0 = g0 - m0 * nchunk;
-            const uint32_t cl = cc0 + lane;
-            const bool next = cl >= nchunk;
-            const uint32_t m = m0 + (next ? 1u : 0u);
-            const uint32_t cc = next ? cl - nchunk : cl;
-            const bool valid = m < static_cast<uint32_t>(M);        // uniform over each block of four lanes
-            float f[8];
-            bf16x8_to_f32(v[u], f);
-            float a = 0.0f;
+        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
+        xq_row[cc] = e2m1x8(g);
+        if ((lane & 3) == 0) xs_row[(blk >> 2) * 512 + (blk & 3)] = static_cast<uint8_t>(E + 127);
+        if (slice_group && cc < nchunk_s) {
+            const int Es = mx_exponent(as);
+            const float invs = mx_inv_scale(Es);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(f[e]));
-            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-            // the salient slice: its own block maximum over the first r columns
-            const bool in_slice = valid && cc < nchunk_s;
-            float as = 0.0f;
-            if (__any_sync(0xFFFFFFFFu, in_slice)) {
-                if (in_slice) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (static_cast<int>(cc) * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
-                }
-                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
-                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
-            }
-            if (!valid) continue;
-            const int blk = static_cast<int>(cc) >> 2;
-            const int E = mx_exponent(a);
-            const float inv = mx_inv_scale(E);
-            float g[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
-            xq[static_cast<size_t>(m) * nchunk + cc] = e2m1x8(g);
+            for (int e = 0; e < 8; ++e) g[e] = (cc * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+            xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
             if ((lane & 3) == 0)
-                xs_atoms[sf_atom_offset(static_cast<int>(m), blk, atoms_k)] = static_cast<uint8_t>(E + 127);
-            if (in_slice) {
-                const int Es = mx_exponent(as);
-                const float invs = mx_inv_scale(Es);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) g[e] = (static_cast<int>(cc) * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
-                xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
-                if ((lane & 3) == 0)
-                    xss_atoms[sf_atom_offset(static_cast<int>(m), blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
-            }
+                xss_atoms[static_cast<size_t>(m >> 7) * atoms_s * 512 + row_sf + (blk >> 2) * 512 + (blk & 3)] =
+                    static_cast<uint8_t>(Es + 127);
         }
     }
 }

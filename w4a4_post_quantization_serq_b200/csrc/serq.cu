@@ -939,15 +939,11 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
                                                                    static_cast<uint32_t*>(xsq),
                                                                    static_cast<float*>(xss));
     } else {
-        // flat stream over the M x K/8 chunks: up to 8 CTAs per SM, each warp
-        // taking 32 * QF_UNROLL chunks per pass (chunk indices are 32-bit)
-        const long long chunks = static_cast<long long>(M) * (K / 8);
-        if (chunks >= (1LL << 31)) return fail(SERQ_EUNSUPPORTED, "M*K=%lld above 2^34", chunks * 8);
-        const long long per_cta = static_cast<long long>(kQuantThreads) * QF_UNROLL;
-        long long grid = (chunks + per_cta - 1) / per_cta;
-        if (grid > 8LL * info->sms) grid = 8LL * info->sms;
-        quant_act_mxfp4_flat_kernel<<<static_cast<unsigned>(grid), kQuantThreads, 0, cs>>>(
-            X, M, K, r, rp, static_cast<uint32_t*>(xq), static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
+        // a CTA per segment of QF_CHUNKS 16-byte chunks of one row
+        if (M > 65535) return fail(SERQ_EUNSUPPORTED, "M=%d above 65535", M);
+        const dim3 grid((K / 8 + QF_CHUNKS - 1) / QF_CHUNKS, M);
+        quant_act_mxfp4_flat_kernel<<<grid, QF_THREADS, 0, cs>>>(
+            X, K, r, rp, static_cast<uint32_t*>(xq), static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
             static_cast<uint8_t*>(xss));
     }
     SERQ_CUDA(cudaGetLastError());
