@@ -21,11 +21,9 @@
 //    and the two forms agree bit for bit;
 //  * programmatic dependent launch: after its set-up each CTA lets the next
 //    kernel of the stream start, and the weight tiles of the first stages are
-//    requested before waiting for the preceding kernel (the tiles past the
-//    ring are prefetched into L2 at the same time, so later refills wait on
-//    L2, not HBM); token data is read, and the workspace and Y are written,
-//    only after that wait. Weight streaming of consecutive linears thus
-//    overlaps the previous one's tail.
+//    requested before waiting for the preceding kernel; token data is read,
+//    and the workspace and Y are written, only after that wait. Weight
+//    streaming of consecutive linears thus overlaps the previous one's tail.
 #pragma once
 
 #include <cstdint>
@@ -145,17 +143,6 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
                 bulk_load(sSFA + i * SFA_BYTES,
                           (res ? p.sf_wr : p.sf_w) + (static_cast<size_t>(n_blk) * atoms + 2 * kk) * 512, na * 512,
                           &full[i]);
-            }
-            // the weight tiles past the ring go to L2 now, so their stage refills later
-            // wait for L2 rather than HBM
-            for (int kt = kt0 + pre; kt < kt1; ++kt) {
-                const bool res = kt >= p.k_tiles_main;
-                const int kk = res ? kt - p.k_tiles_main : kt;
-                const int atoms = res ? p.atoms_k_res : p.atoms_k_main;
-                const int na = min(2, atoms - 2 * kk);
-                tma_prefetch_l2_2d(res ? &tm_wr : &tm_w, kk * BK_BYTES, n_blk * BM);
-                bulk_prefetch_l2((res ? p.sf_wr : p.sf_w) + (static_cast<size_t>(n_blk) * atoms + 2 * kk) * 512,
-                                 na * 512);
             }
             pdl_wait_prerequisites();
             int s = 0;
