@@ -115,6 +115,9 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
         mbar_init(acc_full, 1);
         mbar_init(drain, 1);
         fence_mbar_init();
+        // the token maps are first used right after the wait on the preceding kernel
+        tma_prefetch_desc(&tm_x);
+        if (p.k_tiles_total > p.k_tiles_main) tma_prefetch_desc(&tm_xr);
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, TMEM_COLS);

@@ -227,6 +227,46 @@ __device__ __forceinline__ void quant_row_int8(const Src& src, int m, int K, int
     }
 }
 
+// One 16-byte chunk (eight values f, positions 8c..8c+7 of row m) of an MXFP4
+// row: the block maximum over the four lanes that hold the block's chunks
+// (all 32 lanes must call this together), E8M0 exponent, E2M1 codes, and the
+// salient slice's own block inside the first rp columns. Nothing is written
+// for an invalid chunk (its values must be zeros).
+__device__ __forceinline__ void mx_chunk_out(const float (&f)[8], bool valid, int c, int m, int r, int rp, int nchunk,
+                                             uint32_t* __restrict__ xq, uint8_t* __restrict__ xs_atoms,
+                                             uint32_t* __restrict__ xsq, uint8_t* __restrict__ xss_atoms,
+                                             int atoms_k, int atoms_s) {
+    const int nchunk_s = rp >> 3;
+    float a = 0.0f, as = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+        a = fmaxf(a, fabsf(f[e]));
+        if (c * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
+    }
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+    a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+    as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+    as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+    if (!valid) return;
+    const int blk = c >> 2;
+    const int E = mx_exponent(a);
+    const float inv = mx_inv_scale(E);
+    float g[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
+    xq[static_cast<size_t>(m) * nchunk + c] = e2m1x8(g);
+    if ((threadIdx.x & 3) == 0) xs_atoms[sf_atom_offset(m, blk, atoms_k)] = static_cast<uint8_t>(E + 127);
+    if (c < nchunk_s) {
+        // the slice's own block over its first r columns (zeros beyond r)
+        const int Es = mx_exponent(as);
+        const float invs = mx_inv_scale(Es);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) g[e] = (c * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+        xsq[static_cast<size_t>(m) * nchunk_s + c] = e2m1x8(g);
+        if ((threadIdx.x & 3) == 0) xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
+    }
+}
+
 // MXFP4, one CTA per row; four consecutive threads share one 32-element block.
 template <class Src>
 __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, int r, int rp,
@@ -234,7 +274,6 @@ __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, in
                                                 uint32_t* __restrict__ xsq, uint8_t* __restrict__ xss_atoms) {
     const int nchunk = K >> 3;
     const int atoms_k = (K / 32 + 3) / 4;
-    const int nchunk_s = rp >> 3;
     const int atoms_s = (rp / 32 + 3) / 4;
     const int iters = (nchunk + kQuantThreads - 1) / kQuantThreads;
     for (int j = 0; j < iters; ++j) {
@@ -247,36 +286,7 @@ __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, in
 #pragma unroll
             for (int e = 0; e < 8; ++e) f[e] = 0.0f;
         }
-        float a = 0.0f, as = 0.0f;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            a = fmaxf(a, fabsf(f[e]));
-            if (c * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
-        }
-        // the four chunks of a block sit in four consecutive lanes
-        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-        as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
-        as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
-        if (!valid) continue;
-        const int blk = c >> 2;
-        const int E = mx_exponent(a);
-        const float inv = mx_inv_scale(E);
-        float g[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
-        xq[static_cast<size_t>(m) * nchunk + c] = e2m1x8(g);
-        if ((threadIdx.x & 3) == 0) xs_atoms[sf_atom_offset(m, blk, atoms_k)] = static_cast<uint8_t>(E + 127);
-        if (c < nchunk_s) {
-            // the slice's own block over its first r columns (zeros beyond r)
-            const int Es = mx_exponent(as);
-            const float invs = mx_inv_scale(Es);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = (c * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
-            xsq[static_cast<size_t>(m) * nchunk_s + c] = e2m1x8(g);
-            if ((threadIdx.x & 3) == 0)
-                xss_atoms[sf_atom_offset(m, blk, atoms_s)] = static_cast<uint8_t>(Es + 127);
-        }
+        mx_chunk_out(f, valid, c, m, r, rp, nchunk, xq, xs_atoms, xsq, xss_atoms, atoms_k, atoms_s);
     }
 }
 
@@ -293,93 +303,82 @@ quant_act_int8_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint8_t
 
 // MXFP4 serq_quant_act as a stream over X^: an MX block (32 values, four
 // 16-byte chunks) needs nothing beyond its own row segment, so no row-wide
-// reduction is needed. Grid (ceil(K/8 / QF_CHUNKS), ceil(M / QF_ROWS)): a CTA
-// owns one segment of QF_CHUNKS chunks of QF_ROWS consecutive rows; each warp
-// takes QF_UNROLL groups of 32 consecutive chunks per row (the four chunks of
-// a block in four consecutive lanes) and issues the loads of all its rows
-// before using any. The row comes from the grid, so the addressing is a few
-// adds; the salient slice is handled only by groups that reach into the first
-// rp columns.
+// reduction is needed. Grid (ceil(K/8 / QF_CHUNKS), M): a CTA owns one
+// segment of QF_CHUNKS chunks of one row, each warp QF_UNROLL groups of 32
+// consecutive chunks (the four chunks of a block in four consecutive lanes),
+// all of its loads issued before any is used. The row is blockIdx.y, so the
+// addressing is a few adds; the salient slice is handled only by groups that
+// reach into the first rp columns.
 constexpr int QF_UNROLL = 4;
-constexpr int QF_ROWS = 4;
 constexpr int QF_THREADS = 128;
 constexpr int QF_CHUNKS = QF_THREADS * QF_UNROLL;  // 512 chunks = 4096 values of a row per CTA
 
 __global__ void __launch_bounds__(QF_THREADS)
-quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int M, int K, int r, int rp, uint32_t* __restrict__ xq,
+quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
                             uint8_t* __restrict__ xs_atoms, uint32_t* __restrict__ xsq,
                             uint8_t* __restrict__ xss_atoms) {
     pdl_launch_dependents();  // a programmatically launched consumer waits for this grid before reading
     const int nchunk = K >> 3;
     const int nchunk_s = rp >> 3;
-    const int m0 = blockIdx.y * QF_ROWS;
+    const int m = blockIdx.y;
     const int lane = threadIdx.x & 31;
     const int c_base = blockIdx.x * QF_CHUNKS + (threadIdx.x >> 5) * (32 * QF_UNROLL);
-    uint4 v[QF_ROWS][QF_UNROLL];
+    const uint4* row = X + static_cast<size_t>(m) * nchunk;
+    uint4 v[QF_UNROLL];
 #pragma unroll
-    for (int i = 0; i < QF_ROWS; ++i) {
-        const bool row_ok = m0 + i < M;
-        const uint4* row = X + static_cast<size_t>(row_ok ? m0 + i : 0) * nchunk;
-#pragma unroll
-        for (int u = 0; u < QF_UNROLL; ++u) {
-            const int cc = c_base + u * 32 + lane;
-            v[i][u] = (row_ok && cc < nchunk) ? __ldcs(row + cc) : make_uint4(0u, 0u, 0u, 0u);
-        }
+    for (int u = 0; u < QF_UNROLL; ++u) {
+        const int cc = c_base + u * 32 + lane;
+        v[u] = cc < nchunk ? __ldcs(row + cc) : make_uint4(0u, 0u, 0u, 0u);
     }
+    // this row's scale atoms: row part of the offset fixed, block part per lane
     const int atoms_k = (K / 32 + 3) / 4;
     const int atoms_s = (rp / 32 + 3) / 4;
+    const size_t row_sf = static_cast<size_t>(m & 31) * 16 + static_cast<size_t>((m >> 5) & 3) * 4;
+    uint8_t* xs_row = xs_atoms + static_cast<size_t>(m >> 7) * atoms_k * 512 + row_sf;
+    uint32_t* xq_row = xq + static_cast<size_t>(m) * nchunk;
 #pragma unroll
-    for (int i = 0; i < QF_ROWS; ++i) {
-        const int m = m0 + i;
-        if (m >= M) break;                             // CTA-uniform
-        // this row's scale atoms: row part of the offset fixed, block part per lane
-        const size_t row_sf = static_cast<size_t>(m & 31) * 16 + static_cast<size_t>((m >> 5) & 3) * 4;
-        uint8_t* xs_row = xs_atoms + static_cast<size_t>(m >> 7) * atoms_k * 512 + row_sf;
-        uint32_t* xq_row = xq + static_cast<size_t>(m) * nchunk;
+    for (int u = 0; u < QF_UNROLL; ++u) {
+        const int g0 = c_base + u * 32;
+        if (g0 >= nchunk) break;                       // warp-uniform
+        const int cc = g0 + lane;
+        const bool valid = cc < nchunk;                // uniform over each block of four lanes
+        float f[8];
+        bf16x8_to_f32(v[u], f);
+        float a = 0.0f;
 #pragma unroll
-        for (int u = 0; u < QF_UNROLL; ++u) {
-            const int g0 = c_base + u * 32;
-            if (g0 >= nchunk) break;                   // warp-uniform
-            const int cc = g0 + lane;
-            const bool valid = cc < nchunk;            // uniform over each block of four lanes
-            float f[8];
-            bf16x8_to_f32(v[i][u], f);
-            float a = 0.0f;
+        for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(f[e]));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
+        a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
+        // the salient slice: its own block maximum over the first r columns
+        const bool slice_group = g0 < nchunk_s;       // warp-uniform (nchunk_s is a multiple of 8)
+        float as = 0.0f;
+        if (slice_group) {
+            if (valid && cc < nchunk_s) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) a = fmaxf(a, fabsf(f[e]));
-            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-            a = fmaxf(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-            // the salient slice: its own block maximum over the first r columns
-            const bool slice_group = g0 < nchunk_s;   // warp-uniform (nchunk_s is a multiple of 8)
-            float as = 0.0f;
-            if (slice_group) {
-                if (valid && cc < nchunk_s) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (cc * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
-                }
-                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
-                as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+                for (int e = 0; e < 8; ++e)
+                    if (cc * 8 + e < r) as = fmaxf(as, fabsf(f[e]));
             }
-            if (!valid) continue;
-            const int blk = cc >> 2;
-            const int E = mx_exponent(a);
-            const float inv = mx_inv_scale(E);
-            float g[8];
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 1));
+            as = fmaxf(as, __shfl_xor_sync(0xFFFFFFFFu, as, 2));
+        }
+        if (!valid) continue;
+        const int blk = cc >> 2;
+        const int E = mx_exponent(a);
+        const float inv = mx_inv_scale(E);
+        float g[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
-            xq_row[cc] = e2m1x8(g);
-            if ((lane & 3) == 0) xs_row[(blk >> 2) * 512 + (blk & 3)] = static_cast<uint8_t>(E + 127);
-            if (slice_group && cc < nchunk_s) {
-                const int Es = mx_exponent(as);
-                const float invs = mx_inv_scale(Es);
+        for (int e = 0; e < 8; ++e) g[e] = __fmul_rn(f[e], inv);
+        xq_row[cc] = e2m1x8(g);
+        if ((lane & 3) == 0) xs_row[(blk >> 2) * 512 + (blk & 3)] = static_cast<uint8_t>(E + 127);
+        if (slice_group && cc < nchunk_s) {
+            const int Es = mx_exponent(as);
+            const float invs = mx_inv_scale(Es);
 #pragma unroll
-                for (int e = 0; e < 8; ++e) g[e] = (cc * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
-                xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
-                if ((lane & 3) == 0)
-                    xss_atoms[static_cast<size_t>(m >> 7) * atoms_s * 512 + row_sf + (blk >> 2) * 512 + (blk & 3)] =
-                        static_cast<uint8_t>(Es + 127);
-            }
+            for (int e = 0; e < 8; ++e) g[e] = (cc * 8 + e < r) ? __fmul_rn(f[e], invs) : 0.0f;
+            xsq[static_cast<size_t>(m) * nchunk_s + cc] = e2m1x8(g);
+            if ((lane & 3) == 0)
+                xss_atoms[static_cast<size_t>(m >> 7) * atoms_s * 512 + row_sf + (blk >> 2) * 512 + (blk & 3)] =
+                    static_cast<uint8_t>(Es + 127);
         }
     }
 }

@@ -939,11 +939,11 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
                                                                    static_cast<uint32_t*>(xsq),
                                                                    static_cast<float*>(xss));
     } else {
-        // a CTA per segment of QF_CHUNKS 16-byte chunks of QF_ROWS rows
-        const dim3 grid((K / 8 + QF_CHUNKS - 1) / QF_CHUNKS, (M + QF_ROWS - 1) / QF_ROWS);
-        if (grid.y > 65535u) return fail(SERQ_EUNSUPPORTED, "M=%d above %d", M, 65535 * QF_ROWS);
+        // a CTA per segment of QF_CHUNKS 16-byte chunks of one row
+        if (M > 65535) return fail(SERQ_EUNSUPPORTED, "M=%d above 65535", M);
+        const dim3 grid((K / 8 + QF_CHUNKS - 1) / QF_CHUNKS, M);
         quant_act_mxfp4_flat_kernel<<<grid, QF_THREADS, 0, cs>>>(
-            X, M, K, r, rp, static_cast<uint32_t*>(xq), static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
+            X, K, r, rp, static_cast<uint32_t*>(xq), static_cast<uint8_t*>(xs), static_cast<uint32_t*>(xsq),
             static_cast<uint8_t*>(xss));
     }
     SERQ_CUDA(cudaGetLastError());
