@@ -20,6 +20,8 @@
 namespace serq {
 
 constexpr int kQuantThreads = 256;
+constexpr int kInt4Max = 7;     // INT4 activation codes: s = max|x| / 7
+constexpr int kInt8Max = 127;   // INT8 (W4A8) activation codes: s = max|x| / 127
 
 __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
     const uint32_t w[4] = {v.x, v.y, v.z, v.w};
@@ -30,7 +32,29 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
     }
 }
 
+// rint(fl(x / s)) (IEEE division, ties to even) for |x / s| <= 128, dividing
+// only near a tie: q = fl(x * fl(1/s)) is within 2^-22 |x / s| (< 4e-5) of
+// x / s, so when q is farther than 1e-4 from every half-integer, fl(x / s)
+// lies on the same side of it and rounds to the same integer. (inv_s = inf
+// or a NaN q fails the test and takes the division.)
+__device__ __noinline__ float rint_div(float x, float s) { return rintf(__fdiv_rn(x, s)); }
+
+__device__ __forceinline__ float rint_quot(float x, float s, float inv_s) {
+    const float q = __fmul_rn(x, inv_s);
+    if (fabsf(fabsf(q - truncf(q)) - 0.5f) > 1e-4f) return rintf(q);
+    return rint_div(x, s);  // rare: kept out of line
+}
+
 // INT4 code of x under scale s (two's complement nibble); 0 when s == 0.
+// |x| <= the absmax s was taken from, so |x / s| <= 7 (1 + 2^-23).
+__device__ __forceinline__ uint32_t int4_code(float x, float s, float inv_s) {
+    if (!(s > 0.0f)) return 0u;
+    float q = rint_quot(x, s, inv_s);
+    q = fminf(fmaxf(q, -7.0f), 7.0f);
+    return static_cast<uint32_t>(static_cast<int>(q)) & 0xFu;
+}
+
+// The same with the division always taken (the offline weight quantizers).
 __device__ __forceinline__ uint32_t int4_code(float x, float s) {
     if (!(s > 0.0f)) return 0u;
     float q = rintf(__fdiv_rn(x, s));
@@ -134,6 +158,7 @@ __device__ __forceinline__ void quant_row_int4(const Src& src, int m, int K, int
     block_max2(amax, amax_s, red);
     const float s = __fdiv_rn(amax, 7.0f);
     const float ss = __fdiv_rn(amax_s, 7.0f);
+    const float inv = __fdiv_rn(1.0f, s), invs = __fdiv_rn(1.0f, ss);
     if (threadIdx.x == 0) {
         xs[m] = s;
         if (rp > 0) xss[m] = ss;
@@ -147,13 +172,13 @@ __device__ __forceinline__ void quant_row_int4(const Src& src, int m, int K, int
             bf16x8_to_f32(v[j], f);
             uint32_t w = 0;
 #pragma unroll
-            for (int e = 0; e < 8; ++e) w |= int4_code(f[e], s) << (4 * e);
+            for (int e = 0; e < 8; ++e) w |= int4_code(f[e], s, inv) << (4 * e);
             xq[static_cast<size_t>(m) * nchunk + c] = w;
             if (c < nchunk_s) {
                 uint32_t ws = 0;
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    if (c * 8 + e < r) ws |= int4_code(f[e], ss) << (4 * e);
+                    if (c * 8 + e < r) ws |= int4_code(f[e], ss, invs) << (4 * e);
                 xsq[static_cast<size_t>(m) * nchunk_s + c] = ws;
             }
         }
@@ -162,9 +187,9 @@ __device__ __forceinline__ void quant_row_int4(const Src& src, int m, int K, int
 
 // INT8 code of x under scale s (the W4A8 activations): clip(rne(x / s), -127, 127)
 // as a byte; 0 when s == 0.
-__device__ __forceinline__ uint32_t int8_code(float x, float s) {
+__device__ __forceinline__ uint32_t int8_code(float x, float s, float inv_s) {
     if (!(s > 0.0f)) return 0u;
-    float q = rintf(__fdiv_rn(x, s));
+    float q = rint_quot(x, s, inv_s);
     q = fminf(fmaxf(q, -127.0f), 127.0f);
     return static_cast<uint32_t>(static_cast<int>(q)) & 0xFFu;
 }
@@ -196,6 +221,7 @@ __device__ __forceinline__ void quant_row_int8(const Src& src, int m, int K, int
     block_max2(amax, amax_s, red);
     const float s = __fdiv_rn(amax, 127.0f);
     const float ss = __fdiv_rn(amax_s, 127.0f);
+    const float inv = __fdiv_rn(1.0f, s), invs = __fdiv_rn(1.0f, ss);
     if (threadIdx.x == 0) {
         xs[m] = s;
         if (rp > 0) xss[m] = ss;
@@ -210,16 +236,16 @@ __device__ __forceinline__ void quant_row_int8(const Src& src, int m, int K, int
             uint32_t w0 = 0, w1 = 0;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                w0 |= int8_code(f[e], s) << (8 * e);
-                w1 |= int8_code(f[4 + e], s) << (8 * e);
+                w0 |= int8_code(f[e], s, inv) << (8 * e);
+                w1 |= int8_code(f[4 + e], s, inv) << (8 * e);
             }
             *reinterpret_cast<uint2*>(xq + static_cast<size_t>(m) * K + c * 8) = make_uint2(w0, w1);
             if (c < nchunk_s) {
                 uint32_t s0 = 0, s1 = 0;
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
-                    if (c * 8 + e < r) s0 |= int8_code(f[e], ss) << (8 * e);
-                    if (c * 8 + 4 + e < r) s1 |= int8_code(f[4 + e], ss) << (8 * e);
+                    if (c * 8 + e < r) s0 |= int8_code(f[e], ss, invs) << (8 * e);
+                    if (c * 8 + 4 + e < r) s1 |= int8_code(f[4 + e], ss, invs) << (8 * e);
                 }
                 *reinterpret_cast<uint2*>(xsq + static_cast<size_t>(m) * rp + c * 8) = make_uint2(s0, s1);
             }
@@ -291,7 +317,7 @@ __device__ __forceinline__ void quant_row_mxfp4(const Src& src, int m, int K, in
 }
 
 template <int MAXC>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, MAXC <= 2 ? 8 : 1)
 quant_act_int8_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint8_t* __restrict__ xq,
                       float* __restrict__ xs, uint8_t* __restrict__ xsq, float* __restrict__ xss) {
     __shared__ float red[64];
@@ -385,7 +411,7 @@ quant_act_mxfp4_flat_kernel(const uint4* __restrict__ X, int K, int r, int rp, u
 
 // serq_quant_act: one CTA per token row of X^ (bf16, row-major).
 template <int MAXC>
-__global__ void __launch_bounds__(kQuantThreads)
+__global__ void __launch_bounds__(kQuantThreads, MAXC <= 2 ? 8 : 1)
 quant_act_int4_kernel(const uint4* __restrict__ X, int K, int r, int rp, uint32_t* __restrict__ xq,
                       float* __restrict__ xs, uint32_t* __restrict__ xsq, float* __restrict__ xss) {
     __shared__ float red[64];

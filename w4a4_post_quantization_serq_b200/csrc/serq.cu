@@ -918,26 +918,34 @@ serq_status serq_quant_act(const void* Xhat, int M, int K, int r, int fmt, void*
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
     const int rp = residual_width(r);
     const uint4* X = static_cast<const uint4*>(Xhat);
-    if (fmt == SERQ_FMT_W4A8) {
-        if (K <= 16384)
-            quant_act_int8_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint8_t*>(xq),
-                                                                  static_cast<float*>(xs), static_cast<uint8_t*>(xsq),
-                                                                  static_cast<float*>(xss));
-        else
-            quant_act_int8_kernel<16><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint8_t*>(xq),
-                                                                   static_cast<float*>(xs), static_cast<uint8_t*>(xsq),
-                                                                   static_cast<float*>(xss));
-    } else if (fmt == SERQ_FMT_INT4) {
-        if (K <= 16384)
-            quant_act_int4_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint32_t*>(xq),
-                                                                  static_cast<float*>(xs),
-                                                                  static_cast<uint32_t*>(xsq),
-                                                                  static_cast<float*>(xss));
-        else
-            quant_act_int4_kernel<16><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, static_cast<uint32_t*>(xq),
-                                                                   static_cast<float*>(xs),
-                                                                   static_cast<uint32_t*>(xsq),
-                                                                   static_cast<float*>(xss));
+    if (fmt != SERQ_FMT_MXFP4) {
+        // a CTA per row holding its chunks in registers: the fewest per thread that
+        // cover K, so that short rows take few registers and many rows are in flight
+        const int per_thread = (K / 8 + kQuantThreads - 1) / kQuantThreads;
+        const int maxc = per_thread <= 1 ? 1 : per_thread <= 2 ? 2 : per_thread <= 4 ? 4 : per_thread <= 8 ? 8 : 16;
+        float* fxs = static_cast<float*>(xs);
+        float* fxss = static_cast<float*>(xss);
+        if (fmt == SERQ_FMT_W4A8) {
+            auto* q8 = static_cast<uint8_t*>(xq);
+            auto* qs8 = static_cast<uint8_t*>(xsq);
+            switch (maxc) {
+                case 1: quant_act_int8_kernel<1><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q8, fxs, qs8, fxss); break;
+                case 2: quant_act_int8_kernel<2><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q8, fxs, qs8, fxss); break;
+                case 4: quant_act_int8_kernel<4><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q8, fxs, qs8, fxss); break;
+                case 8: quant_act_int8_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q8, fxs, qs8, fxss); break;
+                default: quant_act_int8_kernel<16><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q8, fxs, qs8, fxss);
+            }
+        } else {
+            auto* q4 = static_cast<uint32_t*>(xq);
+            auto* qs4 = static_cast<uint32_t*>(xsq);
+            switch (maxc) {
+                case 1: quant_act_int4_kernel<1><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q4, fxs, qs4, fxss); break;
+                case 2: quant_act_int4_kernel<2><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q4, fxs, qs4, fxss); break;
+                case 4: quant_act_int4_kernel<4><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q4, fxs, qs4, fxss); break;
+                case 8: quant_act_int4_kernel<8><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q4, fxs, qs4, fxss); break;
+                default: quant_act_int4_kernel<16><<<M, kQuantThreads, 0, cs>>>(X, K, r, rp, q4, fxs, qs4, fxss);
+            }
+        }
     } else {
         // a CTA per segment of QF_CHUNKS 16-byte chunks of one row
         if (M > 65535) return fail(SERQ_EUNSUPPORTED, "M=%d above 65535", M);
