@@ -30,6 +30,8 @@ if ROOT not in sys.path:
 METRIC = "serq_linear TOPS (2·M·N·(K+r)/t) and % of FP4 peak; decode GB/s; overhead vs r=0"
 WORKLOAD = "mlp_mxfp4"
 FP4_OVER_BF16 = 4.0  # nominal dense FP4 / dense BF16 tensor throughput on B200 (9 / 2.25 PFLOP/s)
+INT8_OVER_BF16 = 2.0  # nominal dense INT8 / dense BF16 (4.5 / 2.25)
+INT_KERNEL = "serq_linear_int4_kernel"  # INT4 and W4A8 prefill
 CAPTURED_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 DOMINANT_KERNEL = "serq_linear_mxfp4_pair_kernel"  # M > 128 MXFP4 prefill (CTA pairs)
 
@@ -750,17 +752,19 @@ def main():
     # ~0.16 ms inside a ~0.3 ms step, so the burst (not the seconds-long
     # sustained) GEMM peak is its denominator.
     peaks, peak_src = measured_peaks()
-    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
     dom = max(range(len(layers)), key=lambda i: layers[i]["flops"])
+    mx = layers[dom]["lin"].fmt == "mxfp4"
+    ratio, ratio_name = (FP4_OVER_BF16, "FP4") if mx else (INT8_OVER_BF16, "INT8")
+    peak = peaks["bf16_tflops"] * ratio
     achieved = layers[dom]["flops"] / (gemm_ms[dom] * 1e-3) / 1e12
-    traffic = captured_traffic()
-    roofline = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
-                "frac": achieved / fp4_peak, "traffic": traffic,
-                "kernel": DOMINANT_KERNEL, "launch": layers[dom]["lin"].name,
+    traffic = captured_traffic() if mx else None  # the committed capture is of the CTA-pair kernel
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s" if mx else "TOPS",
+                "frac": achieved / peak, "traffic": traffic,
+                "kernel": DOMINANT_KERNEL if mx else INT_KERNEL, "launch": layers[dom]["lin"].name,
                 "flops_per_launch": layers[dom]["flops"],
                 "peak_source": f"{peak_src} bf16 burst {peaks['bf16_tflops']} TFLOP/s x "
-                               f"{FP4_OVER_BF16:g} (nominal dense FP4/BF16 ratio); of measured",
-                "frac_of_sustained": achieved / (peaks["bf16_tflops_sustained"] * FP4_OVER_BF16),
+                               f"{ratio:g} (nominal dense {ratio_name}/BF16 ratio); of measured",
+                "frac_of_sustained": achieved / (peaks["bf16_tflops_sustained"] * ratio),
                 "quant_act": quant_roofline(layers, quant_ms, peaks["hbm_gbs"]),
                 "per_launch_us": {L["lin"].name: round(t * 1e3, 2) for L, t in zip(layers, gemm_ms)},
                 "all_launches_tflops": sum(L["flops"] for L in layers) / (sum(gemm_ms) * 1e-3) / 1e12,
@@ -768,7 +772,9 @@ def main():
 
     line = {"metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "mxfp4 (e2m1 x e2m1, e8m0 per 32, fp32 accumulate)",
+            "vs_baseline": None,
+            "dtype": "mxfp4 (e2m1 x e2m1, e8m0 per 32, fp32 accumulate)" if mx else
+                     "int4 (s4 x s4 on the int8 path, int32 accumulate)",
             "data": "synthetic",
             "config": {"workload": wl.description, "M": wl.M, "r": 128,
                        "linears": [{"name": L["lin"].name, "K": L["lin"].K, "N": L["lin"].N} for L in layers],

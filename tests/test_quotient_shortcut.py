@@ -1,7 +1,7 @@
 """The INT4 / INT8 activation quantizers on the GPU take rint(fl(x / s)) (IEEE
 division, ties to even, the oracle's decision) as rint(fl(x * fl(1 / s)))
-whenever that product is more than 1e-4 away from a half-integer, and divide
-only otherwise. For |x| <= max|x| = qmax * s the product is within 2^-22 of
+whenever that product is more than 1e-4 away from a half-integer
+(|q - rint(q)| < 0.4999), and divide only otherwise. For |x| <= max|x| = qmax * s the product is within 2^-22 of
 x / s relative, so the two cannot round apart. Checked here in float32 on
 random and exactly-tied quotients over the scale range.
 """
@@ -22,7 +22,7 @@ def test_product_rounds_like_the_quotient_away_from_ties():
             x = np.concatenate([x, (k * np.float32(0.5) * s).astype(np.float32)])  # exact ties
             x = x[np.abs(x) <= amax]
             q = (x * inv).astype(np.float32)
-            fast = np.abs(np.abs(q - np.trunc(q)) - np.float32(0.5)) > np.float32(1e-4)
+            fast = np.abs(q - np.rint(q)) < np.float32(0.4999)
             exact = np.rint((x / s).astype(np.float32))
             assert np.array_equal(np.rint(q[fast]), exact[fast])
             assert np.all(~fast[-5000:] | (np.rint(q[-5000:]) == exact[-5000:]))

@@ -34,14 +34,15 @@ __device__ __forceinline__ void bf16x8_to_f32(const uint4& v, float (&f)[8]) {
 
 // rint(fl(x / s)) (IEEE division, ties to even) for |x / s| <= 128, dividing
 // only near a tie: q = fl(x * fl(1/s)) is within 2^-22 |x / s| (< 4e-5) of
-// x / s, so when q is farther than 1e-4 from every half-integer, fl(x / s)
-// lies on the same side of it and rounds to the same integer. (inv_s = inf
-// or a NaN q fails the test and takes the division.)
+// x / s, so when q is farther than 1e-4 from every half-integer (|q - rint(q)|
+// < 0.4999), fl(x / s) lies on the same side of it and rounds to the same
+// integer. (inv_s = inf or a NaN q fails the test and takes the division.)
 __device__ __noinline__ float rint_div(float x, float s) { return rintf(__fdiv_rn(x, s)); }
 
 __device__ __forceinline__ float rint_quot(float x, float s, float inv_s) {
     const float q = __fmul_rn(x, inv_s);
-    if (fabsf(fabsf(q - truncf(q)) - 0.5f) > 1e-4f) return rintf(q);
+    const float r = rintf(q);
+    if (fabsf(q - r) < 0.4999f) return r;
     return rint_div(x, s);  // rare: kept out of line
 }
 
