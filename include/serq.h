@@ -331,8 +331,10 @@ serq_status serq_fold_quant_act(const serq_weight* w, const void* X, int M, void
  *   O_h = softmax(Q_h K_g^T / sqrt(128) + mask(key > query)) V_g,
  *   g = h / (n_q / n_kv); q [M][ldq] (heads at column h*128), k, v [M][ldkv],
  *   o [M][ldo]; all bf16, 16-byte aligned, leading dimensions multiples of 8.
- *   Warp-level bf16 tensor-core MMAs with fp32 accumulation and an online
- *   softmax (the scores never reach memory).
+ *   tcgen05 bf16 MMAs with fp32 accumulation in tensor memory and an online
+ *   softmax (the scores never reach global memory); V is first transposed
+ *   into stream-ordered device scratch (cudaMallocAsync / cudaFreeAsync on
+ *   `stream`, n_kv * 128 * round_up(M, 64) bf16).
  * serq_add: out = bf16(a + b) elementwise over n bf16 values (n % 8 == 0).
  * All asynchronous on `stream`. Errors: EINVAL, EUNSUPPORTED (head_dim), ECUDA.
  * ------------------------------------------------------------------------ */

@@ -1,0 +1,306 @@
+// Causal grouped-query attention for the prefill block (head_dim 128) on the
+// fifth-generation tensor cores: O_h = softmax(Q_h K_g^T / sqrt(d) + causal
+// mask) V_g, g = h / (n_q / n_kv), the standard LLaMA definition.
+//
+// One CTA per (128 queries, head); 64-key tiles in order up to the block's
+// last query. Per key tile j:
+//   S_j = Q K_j^T       tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M = 128,
+//                       N = 64, K = 128, into one of two tensor-memory buffers;
+//   softmax             four warps, one query row per thread (its tensor-memory
+//                       lane): scale, mask, running max m and sum l in the
+//                       exp2 domain, P_j = exp2(S - m) rounded to bf16 into a
+//                       shared-memory tile in the MMA's operand layout;
+//   O_j = P_j V_j       M = 128, N = 128, K = 64, into one of two fp32 buffers;
+//   O += ...            the softmax warps fold O_j into a register
+//                       accumulator with the running-max rescale, while the
+//                       tensor cores work on S_{j+1} and O_{j+1}.
+// Q and K tiles arrive by TMA with the 128-byte swizzle (K-major operands);
+// V enters the second product as its transpose (dims x keys, K-major), which
+// serq_attention_prefill writes first. Warp 0 loads, warp 1 issues the MMAs
+// (one thread) and owns tensor memory, warps 2..5 do the softmax.
+#pragma once
+
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_bf16.h>
+
+#include "ptx.cuh"
+
+namespace serq {
+namespace atc {
+
+constexpr int D = 128;                  // head dimension
+constexpr int BM = 128;                 // queries per CTA: one per tensor-memory lane
+constexpr int BN = 64;                  // keys per tile
+constexpr int STAGES = 3;               // K / V^T tile ring
+constexpr int Q_BYTES = BM * D * 2;     // 32 KB: two column blocks of [128 rows][128 B]
+constexpr int K_BYTES = BN * D * 2;     // 16 KB: two column blocks of [64 rows][128 B]
+constexpr int V_BYTES = D * BN * 2;     // 16 KB: [128 dims][64 keys = 128 B]
+constexpr int P_BYTES = BM * BN * 2;    // 16 KB: [128 queries][64 keys = 128 B]
+constexpr int THREADS = 6 * 32;         // warp 0 TMA, 1 MMA, 2..5 softmax
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t TMEM_S = 0;          // + 64 b: S buffers (64 fp32 columns each)
+constexpr uint32_t TMEM_O = 128;        // + 128 b: O buffers (128 fp32 columns each)
+constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * (K_BYTES + V_BYTES) + 2 * P_BYTES + 256;
+
+}  // namespace atc
+
+// Instruction descriptor of kind::f16 with bf16 operands, fp32 D, both K-major.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
+    return (1u << 4)     // D format: f32
+           | (1u << 7)   // A: bf16
+           | (1u << 10)  // B: bf16
+           | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                            uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+struct AttTcParams {
+    int M, n_q, n_kv;
+    float scale_log2;  // log2(e) / sqrt(d)
+    __nv_bfloat16* o;
+    int ldo;
+};
+
+// V^T of each key-value group: vt[(g * 128 + d) * M_pad + m] = v[m * ldkv + g * 128 + d],
+// zeros for M <= m < M_pad. Tiles of 32 keys x 32 dims through shared memory.
+__global__ void transpose_v_kernel(const __nv_bfloat16* __restrict__ v, int ldkv, int M, int M_pad,
+                                   __nv_bfloat16* __restrict__ vt) {
+    __shared__ __nv_bfloat16 t[32][33];
+    const int k0 = blockIdx.x * 32, d0 = blockIdx.y * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;  // 32 x 8
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int key = k0 + ty + 8 * i;
+        t[ty + 8 * i][tx] = key < M ? v[static_cast<size_t>(key) * ldkv + d0 + tx] : __float2bfloat16(0.0f);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const int d = d0 + ty + 8 * i;
+        if (k0 + tx < M_pad) vt[static_cast<size_t>(d) * M_pad + k0 + tx] = t[tx][ty + 8 * i];
+    }
+}
+
+// grid (ceil(M / 128), n_q): CTA (qb, h) computes queries [128 qb, +128) of head h;
+// blocks taken last-first so the longest (most keys) start first.
+__global__ void __launch_bounds__(atc::THREADS, 1)
+attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_vt, const AttTcParams p) {
+    using namespace atc;
+    extern __shared__ uint8_t smem_atc[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_atc) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = smem;
+    uint8_t* sK = sQ + Q_BYTES;
+    uint8_t* sV = sK + STAGES * K_BYTES;
+    uint8_t* sP = sV + STAGES * V_BYTES;
+    uint64_t* q_full = reinterpret_cast<uint64_t*>(sP + 2 * P_BYTES);
+    uint64_t* kv_full = q_full + 1;         // [STAGES]
+    uint64_t* kv_empty = kv_full + STAGES;  // [STAGES] (MMA commit)
+    uint64_t* s_full = kv_empty + STAGES;   // [2] S_j in tensor memory (MMA commit)
+    uint64_t* s_empty = s_full + 2;         // [2] the softmax warps have read S_j
+    uint64_t* p_full = s_empty + 2;         // [2] P_j in shared memory
+    uint64_t* o_full = p_full + 2;          // [2] O_j in tensor memory (MMA commit)
+    uint64_t* o_empty = o_full + 2;         // [2] the softmax warps have read O_j
+    uint64_t* drain = o_empty + 2;          // every MMA finished (before tensor memory is freed)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int qb = static_cast<int>(gridDim.x) - 1 - static_cast<int>(blockIdx.x);
+    const int h = blockIdx.y;
+    const int g = h / (p.n_q / p.n_kv);
+    const int q0 = qb * BM;
+    const int last_key = min(q0 + BM, p.M);          // keys [0, last_key) can be visible
+    const int n_tiles = (last_key + BN - 1) / BN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(q_full, 1);
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&kv_full[s], 1);
+            mbar_init(&kv_empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&s_full[b], 1);
+            mbar_init(&s_empty[b], 4);
+            mbar_init(&p_full[b], 4);
+            mbar_init(&o_full[b], 1);
+            mbar_init(&o_empty[b], 4);
+        }
+        mbar_init(drain, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+        tma_prefetch_desc(&tm_vt);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ---------------------------------------------------------------- TMA producer
+        if (lane == 0) {
+            mbar_arrive_expect_tx(q_full, Q_BYTES);
+            tma_load_2d(sQ, &tm_q, q_full, (h * D) * 2, q0);
+            tma_load_2d(sQ + Q_BYTES / 2, &tm_q, q_full, (h * D + 64) * 2, q0);
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % STAGES;
+                if (j >= STAGES && !mbar_wait(&kv_empty[s], static_cast<uint32_t>((j / STAGES - 1) & 1), 0x511u))
+                    break;
+                mbar_arrive_expect_tx(&kv_full[s], K_BYTES + V_BYTES);
+                tma_load_2d(sK + s * K_BYTES, &tm_k, &kv_full[s], (g * D) * 2, j * BN);
+                tma_load_2d(sK + s * K_BYTES + K_BYTES / 2, &tm_k, &kv_full[s], (g * D + 64) * 2, j * BN);
+                tma_load_2d(sV + s * V_BYTES, &tm_vt, &kv_full[s], (j * BN) * 2, g * D);
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------------------------------------------------------- MMA issuer
+        if (lane == 0) {
+            const uint32_t id_s = idesc_bf16(BM, BN);
+            const uint32_t id_o = idesc_bf16(BM, D);
+            bool ok = mbar_wait(q_full, 0, 0x521u);
+            auto issue_s = [&](int j) {
+                const int s = j % STAGES, b = j & 1;
+                if (!mbar_wait(&kv_full[s], static_cast<uint32_t>((j / STAGES) & 1), 0x522u)) return false;
+                if (j >= 2 && !mbar_wait(&s_empty[b], static_cast<uint32_t>(((j >> 1) - 1) & 1), 0x523u)) return false;
+                tc_fence_after();
+                const uint32_t q_base = smem_u32(sQ), k_base = smem_u32(sK + s * K_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks) {  // K = 128 dims: 2 column blocks x 4 steps of 16
+                    const int cb = ks >> 2, kk = ks & 3;
+                    tc_mma_bf16(tmem + TMEM_S + 64u * b, sdesc_kmajor_sw128(q_base + cb * (Q_BYTES / 2) + 32 * kk),
+                                sdesc_kmajor_sw128(k_base + cb * (K_BYTES / 2) + 32 * kk), id_s, ks > 0 ? 1u : 0u);
+                }
+                tc_commit(&s_full[b]);
+                return true;
+            };
+            if (ok && n_tiles > 0) ok = issue_s(0);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                if (j + 1 < n_tiles && !issue_s(j + 1)) {
+                    ok = false;
+                    break;
+                }
+                const int b = j & 1, s = j % STAGES;
+                if (!mbar_wait(&p_full[b], static_cast<uint32_t>((j >> 1) & 1), 0x524u) ||
+                    (j >= 2 && !mbar_wait(&o_empty[b], static_cast<uint32_t>(((j >> 1) - 1) & 1), 0x525u))) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t p_base = smem_u32(sP + b * P_BYTES), v_base = smem_u32(sV + s * V_BYTES);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)  // K = 64 keys: 4 steps of 16
+                    tc_mma_bf16(tmem + TMEM_O + 128u * b, sdesc_kmajor_sw128(p_base + 32 * ks),
+                                sdesc_kmajor_sw128(v_base + 32 * ks), id_o, ks > 0 ? 1u : 0u);
+                tc_commit(&o_full[b]);
+                tc_commit(&kv_empty[s]);
+            }
+            tc_commit(drain);
+            mbar_wait(drain, 0, 0x526u);
+        }
+    } else {
+        // ---------------------------------------------------------------- softmax (warps 2..5)
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // query row of this thread = tensor-memory lane
+        const int row = q0 + r;
+        const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+        float o_acc[D];
+#pragma unroll
+        for (int i = 0; i < D; ++i) o_acc[i] = 0.0f;
+        float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+        bool ok = true;
+        // fold O_i (relative to m_i) into the accumulator (relative to m_{i-1}) with alpha_i
+        auto fold_o = [&](int i, float alpha) {
+            const int b = i & 1;
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[b], static_cast<uint32_t>((i >> 1) & 1), 0x532u)) && ok;
+            if (!ok) return;
+            tc_fence_after();
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(t_lane + TMEM_O + 128u * b + 32u * c, v);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) o_acc[32 * c + e] = fmaf(o_acc[32 * c + e], alpha, __uint_as_float(v[e]));
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&o_empty[b]);
+        };
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            const int b = j & 1;
+            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&s_full[b], static_cast<uint32_t>((j >> 1) & 1), 0x531u));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t sv[BN];
+            tmem_ld_32x32b_x32(t_lane + TMEM_S + 64u * b, *reinterpret_cast<uint32_t(*)[32]>(sv));
+            tmem_ld_32x32b_x32(t_lane + TMEM_S + 64u * b + 32u, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+            tmem_ld_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&s_empty[b]);
+            float x[BN];
+            float mt = -INFINITY;
+#pragma unroll
+            for (int e = 0; e < BN; ++e) {
+                const int key = j * BN + e;
+                const float t = key > row ? -INFINITY : __uint_as_float(sv[e]) * p.scale_log2;
+                x[e] = t;
+                mt = fmaxf(mt, t);
+            }
+            const float m_new = fmaxf(m_run, mt);  // finite: key 0 is visible to every row
+            const float alpha = exp2f(m_run - m_new);
+            float sum = 0.0f;
+            uint32_t pw[BN / 2];
+#pragma unroll
+            for (int e = 0; e < BN / 2; ++e) {
+                const float p0 = exp2f(x[2 * e] - m_new), p1 = exp2f(x[2 * e + 1] - m_new);
+                sum += p0 + p1;
+                pw[e] = pack_bf16x2(p0, p1);
+            }
+            l_run = fmaf(l_run, alpha, sum);
+            m_run = m_new;
+            // P_j row r: 64 bf16 = eight 16-byte chunks, chunk c at slot c ^ (r & 7) (128-byte swizzle)
+            const uint32_t prow = smem_u32(sP + b * P_BYTES) + static_cast<uint32_t>(r) * 128u;
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+                st_shared_v4(prow + ((static_cast<uint32_t>(c) ^ (static_cast<uint32_t>(r) & 7u)) << 4), pw[4 * c],
+                             pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&p_full[b]);
+            if (j >= 1) fold_o(j - 1, alpha_prev);
+            alpha_prev = alpha;
+        }
+        if (ok && n_tiles > 0) fold_o(n_tiles - 1, alpha_prev);
+        if (ok && row < p.M) {
+            const float inv = 1.0f / l_run;
+            uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * p.ldo + h * D);
+#pragma unroll
+            for (int c = 0; c < D / 8; ++c)
+                dst[c] = make_uint4(pack_bf16x2(o_acc[8 * c] * inv, o_acc[8 * c + 1] * inv),
+                                    pack_bf16x2(o_acc[8 * c + 2] * inv, o_acc[8 * c + 3] * inv),
+                                    pack_bf16x2(o_acc[8 * c + 4] * inv, o_acc[8 * c + 5] * inv),
+                                    pack_bf16x2(o_acc[8 * c + 6] * inv, o_acc[8 * c + 7] * inv));
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, TMEM_COLS);
+}
+
+}  // namespace serq

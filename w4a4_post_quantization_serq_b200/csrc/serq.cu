@@ -20,6 +20,7 @@
 #include "quant_act.cuh"
 #include "producer.cuh"
 #include "block.cuh"
+#include "attention_tc.cuh"
 #include "prepare.cuh"
 #include "gemm_mxfp4.cuh"
 #include "gemm_int4.cuh"
@@ -1145,7 +1146,7 @@ serq_status serq_rope(void* x, int M, int ld, int n_heads, int head_dim, float b
 serq_status serq_attention_prefill(const void* q, int ldq, const void* k, const void* v, int ldkv, int M, int n_q,
                                    int n_kv, int head_dim, void* o, int ldo, serq_stream stream) {
     if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return fail(SERQ_EINVAL, "NULL pointer");
-    if (head_dim != att::D) return fail(SERQ_EUNSUPPORTED, "head_dim %d (only %d)", head_dim, att::D);
+    if (head_dim != atc::D) return fail(SERQ_EUNSUPPORTED, "head_dim %d (only %d)", head_dim, atc::D);
     if (M < 1 || n_q < 1 || n_kv < 1 || n_q % n_kv != 0) return fail(SERQ_EINVAL, "bad M / head counts");
     if (ldq < n_q * head_dim || ldkv < n_kv * head_dim || ldo < n_q * head_dim || ldq % 8 || ldkv % 8 || ldo % 8)
         return fail(SERQ_EINVAL, "leading dimensions must cover the heads and be multiples of 8");
@@ -1154,15 +1155,40 @@ serq_status serq_attention_prefill(const void* q, int ldq, const void* k, const 
     int dev;
     DeviceInfo* info;
     if (serq_status st = device_check(&dev, &info)) return st;
-    SERQ_CUDA(cudaFuncSetAttribute(attention_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                   att::SMEM_BYTES));
+    SERQ_CUDA(cudaFuncSetAttribute(attention_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   atc::SMEM_BYTES));
     cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
-    const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
-    attention_prefill_kernel<<<dim3((M + att::BM - 1) / att::BM, n_q), att::THREADS, att::SMEM_BYTES, cs>>>(
-        static_cast<const __nv_bfloat16*>(q), ldq, static_cast<const __nv_bfloat16*>(k),
-        static_cast<const __nv_bfloat16*>(v), ldkv, M, n_q, n_kv, scale_log2, static_cast<__nv_bfloat16*>(o), ldo);
-    SERQ_CUDA(cudaGetLastError());
-    return SERQ_OK;
+    // V^T of each key-value group (dims x keys), the second product's K-major B operand;
+    // stream-ordered scratch
+    const int M_pad = (M + 63) / 64 * 64;
+    const size_t vt_bytes = static_cast<size_t>(n_kv) * head_dim * M_pad * sizeof(__nv_bfloat16);
+    void* vt = nullptr;
+    SERQ_CUDA(cudaMallocAsync(&vt, vt_bytes, cs));
+    transpose_v_kernel<<<dim3(M_pad / 32, n_kv * head_dim / 32), dim3(32, 8), 0, cs>>>(
+        static_cast<const __nv_bfloat16*>(v), ldkv, M, M_pad, static_cast<__nv_bfloat16*>(vt));
+    serq_status st = SERQ_OK;
+    const cudaError_t le = cudaGetLastError();
+    if (le != cudaSuccess) st = cuda_fail(le, "transpose_v_kernel");
+    CUtensorMap tm_q, tm_k, tm_vt;
+    if (!st) st = make_map(&tm_q, q, static_cast<uint64_t>(ldq) * 2, M, 128, atc::BM, true);
+    if (!st) st = make_map(&tm_k, k, static_cast<uint64_t>(ldkv) * 2, M, 128, atc::BN, true);
+    if (!st) st = make_map(&tm_vt, vt, static_cast<uint64_t>(M_pad) * 2, static_cast<uint64_t>(n_kv) * head_dim, 128, atc::D, true);
+    if (!st) {
+        AttTcParams p;
+        p.M = M;
+        p.n_q = n_q;
+        p.n_kv = n_kv;
+        p.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(head_dim));
+        p.o = static_cast<__nv_bfloat16*>(o);
+        p.ldo = ldo;
+        attention_tc_kernel<<<dim3((M + atc::BM - 1) / atc::BM, n_q), atc::THREADS, atc::SMEM_BYTES, cs>>>(tm_q, tm_k,
+                                                                                                       tm_vt, p);
+        const cudaError_t ke = cudaGetLastError();
+        if (ke != cudaSuccess) st = cuda_fail(ke, "attention_tc_kernel");
+    }
+    const cudaError_t fe = cudaFreeAsync(vt, cs);
+    if (!st && fe != cudaSuccess) st = cuda_fail(fe, "cudaFreeAsync");
+    return st;
 }
 
 serq_status serq_add(const void* a, const void* b, void* out, size_t n, serq_stream stream) {
