@@ -333,8 +333,9 @@ serq_status serq_fold_quant_act(const serq_weight* w, const void* X, int M, void
  *   o [M][ldo]; all bf16, 16-byte aligned, leading dimensions multiples of 8.
  *   tcgen05 bf16 MMAs with fp32 accumulation in tensor memory and an online
  *   softmax (the scores never reach global memory); V is first transposed
- *   into stream-ordered device scratch (cudaMallocAsync / cudaFreeAsync on
- *   `stream`, n_kv * 128 * round_up(M, 64) bf16).
+ *   into stream-ordered device scratch (n_kv * 128 * round_up(M, 64) bf16,
+ *   allocated and freed on `stream` from a memory pool of the library's that
+ *   keeps what it has grown to).
  * serq_add: out = bf16(a + b) elementwise over n bf16 values (n % 8 == 0).
  * All asynchronous on `stream`. Errors: EINVAL, EUNSUPPORTED (head_dim), ECUDA.
  * ------------------------------------------------------------------------ */

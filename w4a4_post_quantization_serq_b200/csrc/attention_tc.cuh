@@ -10,10 +10,14 @@
 //                       lane): scale, mask, running max m and sum l in the
 //                       exp2 domain, P_j = exp2(S - m) rounded to bf16 into a
 //                       shared-memory tile in the MMA's operand layout;
-//   O_j = P_j V_j       M = 128, N = 128, K = 64, into one of two fp32 buffers;
-//   O += ...            the softmax warps fold O_j into a register
-//                       accumulator with the running-max rescale, while the
-//                       tensor cores work on S_{j+1} and O_{j+1}.
+//   O += P_j V_j        M = 128, N = 128, K = 64, accumulated by the tensor
+//                       cores into one fp32 tile in tensor memory.
+// P_j is taken against a per-row reference maximum m_ref that moves only when
+// the row's running maximum exceeds it by more than TAU (log2 units), so P <=
+// 2^TAU. When a row's reference moves, its warp rescales that row of O (and
+// of the running sum) in tensor memory by exp2(old - new) between O += P_{j-1}
+// V_{j-1} and O += P_j V_j; otherwise nothing but S and P pass through the
+// softmax warps. At the end O / l is stored as bf16.
 // Q and K tiles arrive by TMA with the 128-byte swizzle (K-major operands);
 // V enters the second product as its transpose (dims x keys, K-major), which
 // serq_attention_prefill writes first. Warp 0 loads, warp 1 issues the MMAs
@@ -40,7 +44,8 @@ constexpr int P_BYTES = BM * BN * 2;    // 16 KB: [128 queries][64 keys = 128 B]
 constexpr int THREADS = 6 * 32;         // warp 0 TMA, 1 MMA, 2..5 softmax
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t TMEM_S = 0;          // + 64 b: S buffers (64 fp32 columns each)
-constexpr uint32_t TMEM_O = 128;        // + 128 b: O buffers (128 fp32 columns each)
+constexpr uint32_t TMEM_O = 128;        // O accumulator (128 fp32 columns)
+constexpr float TAU = 8.0f;             // reference-maximum slack (log2 units): P <= 2^8
 constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * (K_BYTES + V_BYTES) + 2 * P_BYTES + 256;
 
 }  // namespace atc
@@ -62,6 +67,27 @@ __device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t a_desc, ui
         ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
+
+// 2^x on the special-function unit (ex2.approx.ftz; 2^-inf = 0).
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+        "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]), "r"(v[8]), "r"(v[9]),
+        "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]), "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]),
+        "r"(v[19]), "r"(v[20]), "r"(v[21]), "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]),
+        "r"(v[28]), "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st_wait_att() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
 struct AttTcParams {
     int M, n_q, n_kv;
@@ -108,9 +134,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
     uint64_t* s_full = kv_empty + STAGES;   // [2] S_j in tensor memory (MMA commit)
     uint64_t* s_empty = s_full + 2;         // [2] the softmax warps have read S_j
     uint64_t* p_full = s_empty + 2;         // [2] P_j in shared memory
-    uint64_t* o_full = p_full + 2;          // [2] O_j in tensor memory (MMA commit)
-    uint64_t* o_empty = o_full + 2;         // [2] the softmax warps have read O_j
-    uint64_t* drain = o_empty + 2;          // every MMA finished (before tensor memory is freed)
+    uint64_t* o_done = p_full + 2;          // [2] O += P_j V_j finished, by tile parity (MMA commit)
+    uint64_t* drain = o_done + 2;           // every MMA finished (before tensor memory is freed)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -131,8 +156,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             mbar_init(&s_full[b], 1);
             mbar_init(&s_empty[b], 4);
             mbar_init(&p_full[b], 4);
-            mbar_init(&o_full[b], 1);
-            mbar_init(&o_empty[b], 4);
+            mbar_init(&o_done[b], 1);
         }
         mbar_init(drain, 1);
         fence_mbar_init();
@@ -193,8 +217,8 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                     break;
                 }
                 const int b = j & 1, s = j % STAGES;
-                if (!mbar_wait(&p_full[b], static_cast<uint32_t>((j >> 1) & 1), 0x524u) ||
-                    (j >= 2 && !mbar_wait(&o_empty[b], static_cast<uint32_t>(((j >> 1) - 1) & 1), 0x525u))) {
+                // P_j written (and, where a row's reference maximum moved, that row of O rescaled)
+                if (!mbar_wait(&p_full[b], static_cast<uint32_t>((j >> 1) & 1), 0x524u)) {
                     ok = false;
                     break;
                 }
@@ -202,9 +226,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 const uint32_t p_base = smem_u32(sP + b * P_BYTES), v_base = smem_u32(sV + s * V_BYTES);
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)  // K = 64 keys: 4 steps of 16
-                    tc_mma_bf16(tmem + TMEM_O + 128u * b, sdesc_kmajor_sw128(p_base + 32 * ks),
-                                sdesc_kmajor_sw128(v_base + 32 * ks), id_o, ks > 0 ? 1u : 0u);
-                tc_commit(&o_full[b]);
+                    tc_mma_bf16(tmem + TMEM_O, sdesc_kmajor_sw128(p_base + 32 * ks),
+                                sdesc_kmajor_sw128(v_base + 32 * ks), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+                tc_commit(&o_done[b]);
                 tc_commit(&kv_empty[s]);
             }
             tc_commit(drain);
@@ -216,28 +240,12 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
         const int r = quad * 32 + lane;  // query row of this thread = tensor-memory lane
         const int row = q0 + r;
         const uint32_t t_lane = tmem + (static_cast<uint32_t>(quad * 32) << 16);
-        float o_acc[D];
-#pragma unroll
-        for (int i = 0; i < D; ++i) o_acc[i] = 0.0f;
-        float m_run = -INFINITY, l_run = 0.0f, alpha_prev = 0.0f;
+        const float sc = p.scale_log2;
+        float m_ref = -INFINITY, l_run = 0.0f;  // reference maximum (scaled, log2 units), running sum
         bool ok = true;
-        // fold O_i (relative to m_i) into the accumulator (relative to m_{i-1}) with alpha_i
-        auto fold_o = [&](int i, float alpha) {
-            const int b = i & 1;
-            ok = __all_sync(0xFFFFFFFFu, mbar_wait(&o_full[b], static_cast<uint32_t>((i >> 1) & 1), 0x532u)) && ok;
-            if (!ok) return;
-            tc_fence_after();
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-                uint32_t v[32];
-                tmem_ld_32x32b_x32(t_lane + TMEM_O + 128u * b + 32u * c, v);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) o_acc[32 * c + e] = fmaf(o_acc[32 * c + e], alpha, __uint_as_float(v[e]));
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&o_empty[b]);
+        auto wait_o = [&](int i) {  // O += P_i V_i finished
+            return __all_sync(0xFFFFFFFFu,
+                              mbar_wait(&o_done[i & 1], static_cast<uint32_t>((i >> 1) & 1), 0x532u));
         };
         for (int j = 0; ok && j < n_tiles; ++j) {
             const int b = j & 1;
@@ -251,28 +259,54 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&s_empty[b]);
-            float x[BN];
+            // causal mask (only tiles reaching past the block's first query can hide keys)
+            const bool diag = (j + 1) * BN - 1 > q0;
             float mt = -INFINITY;
 #pragma unroll
             for (int e = 0; e < BN; ++e) {
-                const int key = j * BN + e;
-                const float t = key > row ? -INFINITY : __uint_as_float(sv[e]) * p.scale_log2;
-                x[e] = t;
-                mt = fmaxf(mt, t);
+                if (diag && j * BN + e > row) sv[e] = __float_as_uint(-INFINITY);
+                mt = fmaxf(mt, __uint_as_float(sv[e]));
             }
-            const float m_new = fmaxf(m_run, mt);  // finite: key 0 is visible to every row
-            const float alpha = exp2f(m_run - m_new);
+            mt *= sc;  // the row's maximum of this tile, scaled (finite on tile 0: key 0 is visible)
+            const bool grow = mt > m_ref + TAU;
+            if (j == 0) {
+                m_ref = mt;
+            } else if (__any_sync(0xFFFFFFFFu, grow)) {
+                // rows whose maximum moved: rescale their row of O once O += P_{j-1} V_{j-1} is done
+                const float f = grow ? ex2_approx(m_ref - mt) : 1.0f;
+                ok = wait_o(j - 1);
+                if (!ok) break;
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    uint32_t v[32];
+                    tmem_ld_32x32b_x32(t_lane + TMEM_O + 32u * c, v);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+                    tmem_st_32x32b_x32(t_lane + TMEM_O + 32u * c, v);
+                }
+                tmem_st_wait_att();
+                tc_fence_before();
+                l_run *= f;
+                if (grow) m_ref = mt;
+            }
+            // P_j = 2^(S * scale - m_ref) <= 2^TAU, into shared-memory buffer b once O += P_{j-2} V_{j-2} read it
             float sum = 0.0f;
             uint32_t pw[BN / 2];
 #pragma unroll
             for (int e = 0; e < BN / 2; ++e) {
-                const float p0 = exp2f(x[2 * e] - m_new), p1 = exp2f(x[2 * e + 1] - m_new);
+                const float p0 = ex2_approx(fmaf(__uint_as_float(sv[2 * e]), sc, -m_ref));
+                const float p1 = ex2_approx(fmaf(__uint_as_float(sv[2 * e + 1]), sc, -m_ref));
                 sum += p0 + p1;
                 pw[e] = pack_bf16x2(p0, p1);
             }
-            l_run = fmaf(l_run, alpha, sum);
-            m_run = m_new;
-            // P_j row r: 64 bf16 = eight 16-byte chunks, chunk c at slot c ^ (r & 7) (128-byte swizzle)
+            l_run += sum;
+            if (j >= 2) {
+                ok = wait_o(j - 2);
+                if (!ok) break;
+            }
+            // row r: 64 bf16 = eight 16-byte chunks, chunk c at slot c ^ (r & 7) (128-byte swizzle)
             const uint32_t prow = smem_u32(sP + b * P_BYTES) + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
             for (int c = 0; c < 8; ++c)
@@ -281,19 +315,27 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[b]);
-            if (j >= 1) fold_o(j - 1, alpha_prev);
-            alpha_prev = alpha;
         }
-        if (ok && n_tiles > 0) fold_o(n_tiles - 1, alpha_prev);
-        if (ok && row < p.M) {
+        if (ok && n_tiles > 0) ok = wait_o(n_tiles - 1);
+        if (ok) {
+            tc_fence_after();
             const float inv = 1.0f / l_run;
             uint4* dst = reinterpret_cast<uint4*>(p.o + static_cast<size_t>(row) * p.ldo + h * D);
 #pragma unroll
-            for (int c = 0; c < D / 8; ++c)
-                dst[c] = make_uint4(pack_bf16x2(o_acc[8 * c] * inv, o_acc[8 * c + 1] * inv),
-                                    pack_bf16x2(o_acc[8 * c + 2] * inv, o_acc[8 * c + 3] * inv),
-                                    pack_bf16x2(o_acc[8 * c + 4] * inv, o_acc[8 * c + 5] * inv),
-                                    pack_bf16x2(o_acc[8 * c + 6] * inv, o_acc[8 * c + 7] * inv));
+            for (int c = 0; c < D / 32; ++c) {
+                uint32_t v[32];
+                tmem_ld_32x32b_x32(t_lane + TMEM_O + 32u * c, v);
+                tmem_ld_wait();
+                if (row < p.M) {
+#pragma unroll
+                    for (int q = 0; q < 4; ++q)
+                        dst[4 * c + q] = make_uint4(
+                            pack_bf16x2(__uint_as_float(v[8 * q]) * inv, __uint_as_float(v[8 * q + 1]) * inv),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 2]) * inv, __uint_as_float(v[8 * q + 3]) * inv),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 4]) * inv, __uint_as_float(v[8 * q + 5]) * inv),
+                            pack_bf16x2(__uint_as_float(v[8 * q + 6]) * inv, __uint_as_float(v[8 * q + 7]) * inv));
+                }
+            }
         }
     }
 

@@ -80,6 +80,7 @@ struct DeviceInfo {
     bool smem_set_mxp = false;
     bool smem_set_prod = false;
     int pair_clusters = 0;  // co-resident 2-CTA clusters of the pair kernel
+    cudaMemPool_t scratch_pool = nullptr;  // stream-ordered scratch that is kept once grown
 };
 
 // split-K ranges of the small-M kernel. Two CTAs fit per SM. A launch first
@@ -136,6 +137,27 @@ serq_status device_check(int* dev_out, DeviceInfo** info_out) {
     if (d.ok != 1) return fail(SERQ_EUNSUPPORTED, "device %d is not an sm_100 (B200-class) GPU", dev);
     *dev_out = dev;
     *info_out = &d;
+    return SERQ_OK;
+}
+
+// The library's stream-ordered scratch pool of a device (created on first use):
+// memory freed into it stays reserved for the next allocation instead of
+// going back to the driver at each synchronization. The process's default
+// pool is left as it is.
+serq_status scratch_pool(int dev, DeviceInfo* info, cudaMemPool_t* out) {
+    std::lock_guard<std::mutex> lk(g_dev_mu);
+    if (info->scratch_pool == nullptr) {
+        cudaMemPoolProps props = {};
+        props.allocType = cudaMemAllocationTypePinned;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        SERQ_CUDA(cudaMemPoolCreate(&pool, &props));
+        uint64_t keep = ~uint64_t(0);
+        SERQ_CUDA(cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep));
+        info->scratch_pool = pool;
+    }
+    *out = info->scratch_pool;
     return SERQ_OK;
 }
 
@@ -1163,7 +1185,9 @@ serq_status serq_attention_prefill(const void* q, int ldq, const void* k, const 
     const int M_pad = (M + 63) / 64 * 64;
     const size_t vt_bytes = static_cast<size_t>(n_kv) * head_dim * M_pad * sizeof(__nv_bfloat16);
     void* vt = nullptr;
-    SERQ_CUDA(cudaMallocAsync(&vt, vt_bytes, cs));
+    cudaMemPool_t pool;
+    if (serq_status pst = scratch_pool(dev, info, &pool)) return pst;
+    SERQ_CUDA(cudaMallocFromPoolAsync(&vt, vt_bytes, pool, cs));
     transpose_v_kernel<<<dim3(M_pad / 32, n_kv * head_dim / 32), dim3(32, 8), 0, cs>>>(
         static_cast<const __nv_bfloat16*>(v), ldkv, M, M_pad, static_cast<__nv_bfloat16*>(vt));
     serq_status st = SERQ_OK;
