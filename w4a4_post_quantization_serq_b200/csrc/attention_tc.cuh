@@ -2,15 +2,15 @@
 // fifth-generation tensor cores: O_h = softmax(Q_h K_g^T / sqrt(d) + causal
 // mask) V_g, g = h / (n_q / n_kv), the standard LLaMA definition.
 //
-// One CTA per (128 queries, head); 64-key tiles in order up to the block's
+// One CTA per (128 queries, head); 128-key tiles in order up to the block's
 // last query. Per key tile j:
 //   S_j = Q K_j^T       tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M = 128,
-//                       N = 64, K = 128, into one of two tensor-memory buffers;
+//                       N = 128, K = 128, into one of two tensor-memory buffers;
 //   softmax             four warps, one query row per thread (its tensor-memory
 //                       lane): scale, mask, running max m and sum l in the
 //                       exp2 domain, P_j = exp2(S - m) rounded to bf16 into a
 //                       shared-memory tile in the MMA's operand layout;
-//   O += P_j V_j        M = 128, N = 128, K = 64, accumulated by the tensor
+//   O += P_j V_j        M = 128, N = 128, K = 128, accumulated by the tensor
 //                       cores into one fp32 tile in tensor memory.
 // P_j is taken against a per-row reference maximum m_ref that moves only when
 // the row's running maximum exceeds it by more than TAU (log2 units), so P <=
@@ -35,16 +35,18 @@ namespace atc {
 
 constexpr int D = 128;                  // head dimension
 constexpr int BM = 128;                 // queries per CTA: one per tensor-memory lane
-constexpr int BN = 64;                  // keys per tile
-constexpr int STAGES = 3;               // K / V^T tile ring
-constexpr int Q_BYTES = BM * D * 2;     // 32 KB: two column blocks of [128 rows][128 B]
-constexpr int K_BYTES = BN * D * 2;     // 16 KB: two column blocks of [64 rows][128 B]
-constexpr int V_BYTES = D * BN * 2;     // 16 KB: [128 dims][64 keys = 128 B]
-constexpr int P_BYTES = BM * BN * 2;    // 16 KB: [128 queries][64 keys = 128 B]
+constexpr int BN = 128;                 // keys per tile
+constexpr int KB = BN / 64;             // 128-byte column blocks of a key row (P, V^T)
+constexpr int STAGES = 2;               // K / V^T tile ring
+constexpr int Q_BYTES = BM * D * 2;     // 32 KB: two column blocks of [128 queries][128 B]
+constexpr int K_BYTES = BN * D * 2;     // 32 KB: two column blocks of [128 keys][128 B]
+constexpr int V_BYTES = D * BN * 2;     // 32 KB: KB column blocks of [128 dims][64 keys = 128 B]
+constexpr int P_BYTES = BM * BN * 2;    // 32 KB: KB column blocks of [128 queries][64 keys = 128 B]
+constexpr int CB_BYTES = 128 * 128;     // one column block of 128 rows
 constexpr int THREADS = 6 * 32;         // warp 0 TMA, 1 MMA, 2..5 softmax
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t TMEM_S = 0;          // + 64 b: S buffers (64 fp32 columns each)
-constexpr uint32_t TMEM_O = 128;        // O accumulator (128 fp32 columns)
+constexpr uint32_t TMEM_S = 0;          // + BN b: S buffers (BN fp32 columns each)
+constexpr uint32_t TMEM_O = 2 * BN;     // O accumulator (128 fp32 columns)
 constexpr float TAU = 8.0f;             // reference-maximum slack (log2 units): P <= 2^8
 constexpr int SMEM_BYTES = 1024 + Q_BYTES + STAGES * (K_BYTES + V_BYTES) + 2 * P_BYTES + 256;
 
@@ -186,7 +188,9 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 mbar_arrive_expect_tx(&kv_full[s], K_BYTES + V_BYTES);
                 tma_load_2d(sK + s * K_BYTES, &tm_k, &kv_full[s], (g * D) * 2, j * BN);
                 tma_load_2d(sK + s * K_BYTES + K_BYTES / 2, &tm_k, &kv_full[s], (g * D + 64) * 2, j * BN);
-                tma_load_2d(sV + s * V_BYTES, &tm_vt, &kv_full[s], (j * BN) * 2, g * D);
+#pragma unroll
+                for (int kb = 0; kb < KB; ++kb)
+                    tma_load_2d(sV + s * V_BYTES + kb * CB_BYTES, &tm_vt, &kv_full[s], (j * BN + 64 * kb) * 2, g * D);
             }
         }
     } else if (warp == 1) {
@@ -204,7 +208,7 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks) {  // K = 128 dims: 2 column blocks x 4 steps of 16
                     const int cb = ks >> 2, kk = ks & 3;
-                    tc_mma_bf16(tmem + TMEM_S + 64u * b, sdesc_kmajor_sw128(q_base + cb * (Q_BYTES / 2) + 32 * kk),
+                    tc_mma_bf16(tmem + TMEM_S + static_cast<uint32_t>(BN) * b, sdesc_kmajor_sw128(q_base + cb * (Q_BYTES / 2) + 32 * kk),
                                 sdesc_kmajor_sw128(k_base + cb * (K_BYTES / 2) + 32 * kk), id_s, ks > 0 ? 1u : 0u);
                 }
                 tc_commit(&s_full[b]);
@@ -225,9 +229,11 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 tc_fence_after();
                 const uint32_t p_base = smem_u32(sP + b * P_BYTES), v_base = smem_u32(sV + s * V_BYTES);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)  // K = 64 keys: 4 steps of 16
-                    tc_mma_bf16(tmem + TMEM_O, sdesc_kmajor_sw128(p_base + 32 * ks),
-                                sdesc_kmajor_sw128(v_base + 32 * ks), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+                for (int ks = 0; ks < BN / 16; ++ks) {  // K = BN keys: KB column blocks x 4 steps of 16
+                    const int kb = ks >> 2, kk = ks & 3;
+                    tc_mma_bf16(tmem + TMEM_O, sdesc_kmajor_sw128(p_base + kb * CB_BYTES + 32 * kk),
+                                sdesc_kmajor_sw128(v_base + kb * CB_BYTES + 32 * kk), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+                }
                 tc_commit(&o_done[b]);
                 tc_commit(&kv_empty[s]);
             }
@@ -253,8 +259,10 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
             if (!ok) break;
             tc_fence_after();
             uint32_t sv[BN];
-            tmem_ld_32x32b_x32(t_lane + TMEM_S + 64u * b, *reinterpret_cast<uint32_t(*)[32]>(sv));
-            tmem_ld_32x32b_x32(t_lane + TMEM_S + 64u * b + 32u, *reinterpret_cast<uint32_t(*)[32]>(sv + 32));
+#pragma unroll
+            for (int c = 0; c < BN / 32; ++c)
+                tmem_ld_32x32b_x32(t_lane + TMEM_S + static_cast<uint32_t>(BN) * b + 32u * c,
+                                   *reinterpret_cast<uint32_t(*)[32]>(sv + 32 * c));
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
@@ -306,12 +314,14 @@ attention_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_const
                 ok = wait_o(j - 2);
                 if (!ok) break;
             }
-            // row r: 64 bf16 = eight 16-byte chunks, chunk c at slot c ^ (r & 7) (128-byte swizzle)
+            // row r: BN bf16 = BN / 8 chunks of 16 bytes over KB column blocks; chunk cc of a
+            // block at slot cc ^ (r & 7) (128-byte swizzle)
             const uint32_t prow = smem_u32(sP + b * P_BYTES) + static_cast<uint32_t>(r) * 128u;
 #pragma unroll
-            for (int c = 0; c < 8; ++c)
-                st_shared_v4(prow + ((static_cast<uint32_t>(c) ^ (static_cast<uint32_t>(r) & 7u)) << 4), pw[4 * c],
-                             pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
+            for (int c = 0; c < BN / 8; ++c)
+                st_shared_v4(prow + static_cast<uint32_t>((c >> 3) * CB_BYTES) +
+                                 (((static_cast<uint32_t>(c) & 7u) ^ (static_cast<uint32_t>(r) & 7u)) << 4),
+                             pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             fence_proxy_async_smem();  // generic-proxy writes -> visible to the tensor cores
             __syncwarp();
             if (lane == 0) mbar_arrive(&p_full[b]);
