@@ -309,6 +309,46 @@ def time_e2e(layers, steps, warmup, pg=None):
     return start.elapsed_time(end) / steps, h2d, d2h
 
 
+def bench_small_m(tokens=(32, 64, 128), reps: int = 50):
+    """serq_linear for 16 < M <= 128 (the one-CTA tensor-core kernel) on the
+    gate/up shape (K = 4096, N = 2 x 14336, MXFP4, r = 128), one weight, CUDA
+    events over back-to-back launches. At these M the 59 MB weight stream
+    bounds it, so both the TFLOP/s and the weight GB/s are reported."""
+    import torch
+    import w4a4_post_quantization_serq_b200 as S
+    from synth import workload
+    lin = workload("mlp_mxfp4").linears[0]
+    K, N, r = lin.K, lin.N, lin.r
+    rp = ((r + 63) // 64) * 64
+    W = torch.from_numpy(lin.W()).to(torch.bfloat16).cuda()
+    a = S.serq_calib_absmax(torch.from_numpy(lin.X_calib(128)).to(torch.bfloat16).cuda())
+    w = S.serq_prepare(W, r, lin.fmt, act_absmax=a)
+    del W
+    w_bytes = N * K // 2 + N * K // 32 + N * rp // 2 + N * rp // 32
+    peaks = measured_peaks()[0]
+    out = {"K": K, "N": N, "r": r}
+    for M in tokens:
+        qa = S.serq_quant_act(S.serq_fold_producer(w, torch.from_numpy(lin.X(M)).to(torch.bfloat16).cuda()),
+                              r, lin.fmt)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        for _ in range(5):
+            S.serq_linear(w, qa, Y=Y)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(reps):
+            S.serq_linear(w, qa, Y=Y)
+        end.record()
+        torch.cuda.synchronize()
+        us = start.elapsed_time(end) / reps * 1e3
+        tflops = 2.0 * M * N * (K + r) / (us * 1e-6) / 1e12
+        out[f"M{M}"] = {"us": round(us, 2), "TFLOPs": round(tflops, 1),
+                        "frac_fp4": round(tflops / (peaks["bf16_tflops"] * FP4_OVER_BF16), 3),
+                        "weight_GBs": round(w_bytes / (us * 1e-6) / 1e9, 1),
+                        "frac_hbm": round(w_bytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 3)}
+    S.serq_device_status()
+    return out
+
+
 def bench_decode(reps: int = 10, tokens=(1, 4, 16)):
     """HBM-bound small-M serq_linear on the LLaMA-3-8B decode shapes.
 
@@ -843,6 +883,7 @@ def main():
         line["decode"] = dec
         m16 = [v["M16"]["GBs"] for v in dec.values() if isinstance(v, dict) and "M16" in v]
         line["decode_GBs_M16_mean"] = sum(m16) / len(m16)
+        line["small_m"] = bench_small_m()
         line["stack"] = bench_stack()
         line["prefill_block"] = bench_prefill_block()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
