@@ -86,8 +86,10 @@ struct DeviceInfo {
 // split-K ranges of the small-M kernel. Two CTAs fit per SM. A launch first
 // takes one CTA per SM, leaving the other slot to the next launch, whose CTAs
 // then prefetch their weight stages while this one finishes; when a CTA
-// would still have more K-tiles than its ring holds, the launch takes both
-// slots instead (more bytes in flight). At most kMaxDecodeSplits (the
+// would still have more than one K-tile beyond what its ring holds, the
+// launch takes both slots instead (more bytes in flight; one refill per CTA
+// costs less than giving up that overlap: 4096 x 6144 runs 6.9 us with 144
+// CTAs against 10.1 us with 288). At most kMaxDecodeSplits (the
 // portable cluster size), never more than the K-tiles.
 constexpr int kMaxDecodeSplits = mxd::MAX_SPLITS;
 constexpr int kMaxDecodeTokens = 16;
@@ -100,7 +102,7 @@ int decode_splits(int n_blocks, int k_tiles, int sms) {
         return s < 1 ? 1 : s;
     };
     const int s1 = fit(sms);
-    return (k_tiles + s1 - 1) / s1 > mxd::STAGES ? fit(2 * sms) : s1;
+    return (k_tiles + s1 - 1) / s1 > mxd::STAGES + 1 ? fit(2 * sms) : s1;
 }
 
 // One-time per-device set-up of both forms of the small-M kernel.
