@@ -100,3 +100,23 @@ def test_noalloc_rejects_null_and_unaligned(lib):
     assert lib.serq_linear_small_m_noalloc(*ok, 16, 16, None, 16, 16, 16, 16, 16, 16, None) == N.SERQ_EINVAL
     # an unaligned output pointer
     assert lib.serq_linear_small_m_noalloc(*ok, 16, 16, 16, 16, 16, 16, 16, 16, 24, None) == N.SERQ_EINVAL
+
+
+def test_block_entry_points_reject_before_touching_device(lib):
+    # RoPE: NULL / unaligned x, odd head_dim, ld narrower than the heads, base <= 1
+    assert lib.serq_rope(None, 4, 256, 2, 128, ctypes.c_float(10000.0), 0, None) == N.SERQ_EINVAL
+    assert lib.serq_rope(18, 4, 256, 2, 128, ctypes.c_float(10000.0), 0, None) == N.SERQ_EINVAL
+    assert lib.serq_rope(16, 4, 256, 2, 127, ctypes.c_float(10000.0), 0, None) == N.SERQ_EINVAL
+    assert lib.serq_rope(16, 4, 200, 2, 128, ctypes.c_float(10000.0), 0, None) == N.SERQ_EINVAL
+    assert lib.serq_rope(16, 4, 256, 2, 128, ctypes.c_float(1.0), 0, None) == N.SERQ_EINVAL
+    # attention: NULL, head_dim other than 128, heads not grouping, short leading dims, unaligned
+    att = lib.serq_attention_prefill
+    assert att(None, 256, 16, 16, 128, 4, 2, 1, 128, 16, 256, None) == N.SERQ_EINVAL
+    assert att(16, 128, 16, 16, 64, 4, 2, 1, 64, 16, 128, None) == N.SERQ_EUNSUPPORTED
+    assert att(16, 384, 16, 16, 256, 4, 3, 2, 128, 16, 384, None) == N.SERQ_EINVAL
+    assert att(16, 128, 16, 16, 128, 4, 2, 1, 128, 16, 256, None) == N.SERQ_EINVAL
+    assert att(24, 256, 16, 16, 128, 4, 2, 1, 128, 16, 256, None) == N.SERQ_EINVAL
+    # add: n not a multiple of 8, NULL, unaligned
+    assert lib.serq_add(16, 16, 16, 12, None) == N.SERQ_EINVAL
+    assert lib.serq_add(None, 16, 16, 16, None) == N.SERQ_EINVAL
+    assert lib.serq_add(16, 20, 16, 16, None) == N.SERQ_EINVAL
