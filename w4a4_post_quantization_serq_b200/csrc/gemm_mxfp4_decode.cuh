@@ -10,10 +10,15 @@
 //    streams 128 weight rows over its range;
 //  * split reduction, two forms (template flag):
 //    - cluster: the S split CTAs of an output block form one thread-block
-//      cluster (1 x S x 1); each parks its fp32 partial sums in its own
-//      shared memory, and after a cluster barrier CTA c adds, for its 1/S
-//      share of the block's outputs, the S partials read over distributed
-//      shared memory in split order, and writes bf16 Y. No workspace.
+//      cluster (1 x S x 1). CTA c owns the block's output channels
+//      [c R, c R + R) (R = ceil(128 / S) rounded up to 4). Each split sends
+//      its fp32 partial sums of the channels a peer owns straight into that
+//      peer's shared memory (st.async, 16 bytes at a time, counted on the
+//      peer's "received" mbarrier) and stores those it owns itself, so no CTA
+//      waits for its peers except for the partial sums it owns: the owner
+//      adds the S partials in split order and writes bf16 Y. One cluster
+//      barrier, at set-up, makes the peers' mbarriers visible before the
+//      first send. No workspace.
 //    - workspace: each CTA writes its partial sums to a global workspace; the
 //      last CTA of an output block (ticket counter) adds the S partials in
 //      split order, writes bf16 Y and resets the counter for the next call.
@@ -49,8 +54,10 @@ constexpr uint32_t TMEM_COLS = 32;
 constexpr uint32_t TMEM_ACC = 0;                 // 16 fp32 columns (tokens)
 constexpr uint32_t TMEM_SFA = 16;                // 2 atoms x 4 columns
 constexpr uint32_t TMEM_SFB = 24;                // 2 atoms x 4 columns
-constexpr int PART_BYTES = MAX_TOKENS * BM * 4;  // this CTA's fp32 partial sums (cluster form)
 constexpr int MAX_SPLITS = 8;                    // portable cluster size
+// partial sums received by an owner (cluster form): [split][owned channel][token],
+// at most S * R * 16 * 4 bytes over S <= 8 (S = 6: 6 * 24 * 64 = 9216)
+constexpr int PART_BYTES = 9216;
 constexpr int SMEM_BYTES = STAGES * (A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES) + PART_BYTES + 1024 + 256;
 
 }  // namespace mxd
@@ -92,12 +99,13 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     uint8_t* sB = sA + STAGES * A_BYTES;
     uint8_t* sSFA = sB + STAGES * B_BYTES;
     uint8_t* sSFB = sSFA + STAGES * SFA_BYTES;
-    float* spart = reinterpret_cast<float*>(sSFB + STAGES * SFB_BYTES);  // [MAX_TOKENS][BM]
+    float* spart = reinterpret_cast<float*>(sSFB + STAGES * SFB_BYTES);  // [split][rows_per][nt]
     uint64_t* full = reinterpret_cast<uint64_t*>(sSFB + STAGES * SFB_BYTES + PART_BYTES);
     uint64_t* empty = full + STAGES;
     uint64_t* acc_full = empty + STAGES;
     uint64_t* drain = acc_full + 1;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+    uint64_t* recv_full = drain + 1;  // cluster form: every split's partial sums of the owned channels arrived
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(recv_full + 1);
     __shared__ unsigned int s_is_last;
 
     const int warp = threadIdx.x >> 5;
@@ -106,6 +114,11 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     const int split = blockIdx.y;
     const int kt0 = static_cast<int>((static_cast<long long>(p.k_tiles_total) * split) / p.splits);
     const int kt1 = static_cast<int>((static_cast<long long>(p.k_tiles_total) * (split + 1)) / p.splits);
+    // cluster form: the cluster spans the S splits of this block, so the CTA's rank is its split
+    const int rows_per = ((BM + p.splits - 1) / p.splits + 3) & ~3;
+    const int row0 = split * rows_per;
+    const int rows_own = min(BM, row0 + rows_per) - row0;
+    const int nt = p.n_tokens_mma;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
@@ -114,7 +127,10 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
         }
         mbar_init(acc_full, 1);
         mbar_init(drain, 1);
+        if constexpr (kClusterReduce) mbar_init(recv_full, 1);
         fence_mbar_init();
+        if constexpr (kClusterReduce)
+            mbar_arrive_expect_tx(recv_full, static_cast<uint32_t>((p.splits - 1) * rows_own * nt * 4));
         // the token maps are first used right after the wait on the preceding kernel
         tma_prefetch_desc(&tm_x);
         if (p.k_tiles_total > p.k_tiles_main) tma_prefetch_desc(&tm_xr);
@@ -127,6 +143,7 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
+    if constexpr (kClusterReduce) cluster_arrive();  // this CTA's "received" barrier is initialised
     pdl_launch_dependents();
 
     if (warp == 0) {
@@ -229,22 +246,43 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
         const int quad = warp & 3;
         const int n = n_blk * BM + quad * 32 + lane;
         pdl_wait_prerequisites();  // the preceding kernel is done with the workspace and Y
-        if (__all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, 0x321u))) {
+        uint32_t v[16] = {};
+        const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(acc_full, 0, 0x321u));
+        if (got) {
             tc_fence_after();
-            uint32_t v[16];
             tmem_ld_32x32b_x16(tmem + (static_cast<uint32_t>(quad * 32) << 16) + TMEM_ACC, v);
             tmem_ld_wait();
-            if constexpr (kClusterReduce) {
-                const int row = quad * 32 + lane;
+        }
+        if constexpr (kClusterReduce) {
+            // this channel's partial sums (all nt token columns) go to its owner: a
+            // peer's by st.async (even after a timed-out wait, so that the owners'
+            // barriers complete), this CTA's own by plain stores
+            cluster_wait();
+            const int row = quad * 32 + lane;
+            const int owner = row / rows_per;
+            const int slot = ((split * rows_per + row - owner * rows_per) * nt) * 4;  // bytes into spart
+            if (owner == split) {
+                float4* d = reinterpret_cast<float4*>(reinterpret_cast<uint8_t*>(spart) + slot);
 #pragma unroll
-                for (int m = 0; m < MAX_TOKENS; ++m)
-                    if (m < p.M) spart[m * BM + row] = __uint_as_float(v[m]);
+                for (int j = 0; j < MAX_TOKENS / 4; ++j)
+                    if (4 * j < nt)
+                        d[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                           __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
             } else {
-                float* part = p.partial + static_cast<size_t>(split) * p.M * p.N;
+                const uint32_t dst = mapa_shared(smem_u32(spart) + static_cast<uint32_t>(slot),
+                                                 static_cast<uint32_t>(owner));
+                const uint32_t bar = mapa_shared(smem_u32(recv_full), static_cast<uint32_t>(owner));
 #pragma unroll
-                for (int m = 0; m < MAX_TOKENS; ++m)
-                    if (m < p.M) part[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[m]);
+                for (int j = 0; j < MAX_TOKENS / 4; ++j)
+                    if (4 * j < nt)
+                        st_async_v4f32(dst + 16u * j, __uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                       __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]), bar);
             }
+        } else if (got) {
+            float* part = p.partial + static_cast<size_t>(split) * p.M * p.N;
+#pragma unroll
+            for (int m = 0; m < MAX_TOKENS; ++m)
+                if (m < p.M) part[static_cast<size_t>(m) * p.N + n] = __uint_as_float(v[m]);
         }
         tc_fence_before();
     }
@@ -252,37 +290,32 @@ serq_linear_mxfp4_decode_kernel(const __grid_constant__ CUtensorMap tm_w, const 
     // ---------------------------------------------------------------- split reduction
     pdl_wait_prerequisites();
     if constexpr (kClusterReduce) {
-        __syncwarp();
-        cluster_sync();  // every split's partial sums are in its CTA's shared memory
-        const uint32_t rank = cluster_ctarank();  // == split: the cluster spans the S splits of this block
-        const int total = p.M * (BM / 4);              // groups of 4 consecutive outputs
-        const int chunk = (total + p.splits - 1) / p.splits;
-        const int lo = static_cast<int>(rank) * chunk;
-        const int hi = min(total, lo + chunk);
-        const uint32_t local = smem_u32(spart);
-        for (int g = lo + static_cast<int>(threadIdx.x); g < hi; g += blockDim.x) {
-            float4 part[MAX_SPLITS];
-#pragma unroll
-            for (int sp = 0; sp < MAX_SPLITS; ++sp)
-                if (sp < p.splits) part[sp] = ld_shared_cluster_v4f32(mapa_shared(local + 16u * g, sp));
-            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-#pragma unroll
-            for (int sp = 0; sp < MAX_SPLITS; ++sp) {
-                if (sp < p.splits) {
-                    acc.x += part[sp].x;
-                    acc.y += part[sp].y;
-                    acc.z += part[sp].z;
-                    acc.w += part[sp].w;
-                }
-            }
-            const int m = g / (BM / 4);
-            const int n = n_blk * BM + (g % (BM / 4)) * 4;
-            uint2 out;
-            out.x = pack_bf16x2(acc.x, acc.y);
-            out.y = pack_bf16x2(acc.z, acc.w);
-            *reinterpret_cast<uint2*>(p.Y + static_cast<size_t>(m) * p.N + n) = out;
+        if (warp < 2) {
+            __syncwarp();
+            cluster_wait();  // the epilogue warps waited before their sends
         }
-        cluster_sync();  // no CTA leaves while a peer still reads its partial sums
+        __syncthreads();  // this CTA's own partial sums are in shared memory
+        // then the peers' (counted on recv_full); no peer writes this CTA's shared
+        // memory after that, so it may leave once it has added them
+        if (mbar_wait_cluster(recv_full, 0, 0x323u)) {
+            const int groups = p.M * (rows_own / 4);  // (token, 4 consecutive owned channels)
+            for (int g = threadIdx.x; g < groups; g += blockDim.x) {
+                const int m = g % p.M;
+                const int c = 4 * (g / p.M);
+                float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+                for (int sp = 0; sp < p.splits; ++sp) {
+                    const float* src = spart + (sp * rows_per + c) * nt + m;
+                    acc.x += src[0];
+                    acc.y += src[nt];
+                    acc.z += src[2 * nt];
+                    acc.w += src[3 * nt];
+                }
+                uint2 out;
+                out.x = pack_bf16x2(acc.x, acc.y);
+                out.y = pack_bf16x2(acc.z, acc.w);
+                *reinterpret_cast<uint2*>(p.Y + static_cast<size_t>(m) * p.N + n_blk * BM + row0 + c) = out;
+            }
+        }
     } else {
         __threadfence();
         __syncthreads();
