@@ -42,7 +42,7 @@ RMS_CASES = [("int4", 64, 256, 256, 16), ("mxfp4", 64, 256, 256, 16), ("w4a8", 6
              ("w4a8", 65, 20480, 128, 40), ("int4", 77, 384, 256, 40),
              ("mxfp4", 77, 384, 256, 40), ("mxfp4", 5, 1024, 512, 0), ("int4", 33, 20480, 128, 128),
              ("mxfp4", 129, 4096, 256, 128),
-             ("mxfp4", 1300, 1024, 256, 40),     # several rows per CTA of the persistent kernel
+             ("mxfp4", 1300, 1024, 256, 40),     # many rows, each shorter than the 512 chunks a CTA covers
              ("mxfp4", 40, 32768, 128, 128)]     # too wide to stage two rows: one row per CTA
 
 
